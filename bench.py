@@ -1,0 +1,360 @@
+#!/usr/bin/env python
+"""Decode-step benchmark: single-token MLRA-4 decode over a latent KV cache on B200.
+
+A step is one whole decode call (absorb_q -> split-KV decode -> combine/up-projection)
+over one batch of the workload; inputs are resident in HBM when the timed region
+starts.  Default workload: MLRA-4, B=64, h=128, T=32768, 64-token pages with a random
+page table (2.4 GB of KV cache read per step, larger than L2, so no flush is needed).
+
+    python bench.py [--gpus N --steps K --warmup W] [--workload NAME] [--impl reference]
+
+Multi-GPU (torchrun, one rank per GPU): every rank decodes its own replica batch (the
+path has no exchange step); value = all ranks' KV bytes / max-over-ranks step time.
+One JSON line is printed by rank 0.
+"""
+from __future__ import annotations
+
+import argparse
+import ctypes
+import datetime
+import hashlib
+import json
+import math
+import os
+import pathlib
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = pathlib.Path(__file__).resolve().parent
+sys.path.insert(0, str(ROOT))
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+import synth  # noqa: E402
+
+METRIC = "MLRA-4 decode µs/step & KV-cache read TB/s (fraction of ~8 TB/s HBM)"
+NOMINAL_HBM_GBS = 8000.0
+FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0}
+DECODE_SOURCES = ["head_rank_attention_b200/csrc/decode_sm100.cu", "head_rank_attention_b200/csrc/sm100.cuh",
+                  "head_rank_attention_b200/csrc/schedule.cuh", "head_rank_attention_b200/csrc/decode_sm100.h"]
+
+
+def tensor_flops_per_token(n_branch: int, heads: int) -> int:
+    """Tensor-core FLOPs per cached token the decode kernel issues: each of the 4 slice
+    CTAs scores over its branch (w + 64 dims) for 128 padded head rows, and P.V adds
+    2*512 per head row.  Algorithmic count (shared rope scored once, real heads only):
+    2*(512+64)*h + 2*512*h."""
+    return 2 * (512 + 64) * heads + 2 * 512 * heads
+
+
+def peaks():
+    p = ROOT / "MEASURED_PEAKS.json"
+    if p.exists():
+        d = json.loads(p.read_text())
+        return d, "measured"
+    return dict(FALLBACK), "fallback"
+
+
+def decode_source_hash() -> str:
+    h = hashlib.sha256()
+    for f in DECODE_SOURCES:
+        h.update((ROOT / f).read_bytes())
+    return h.hexdigest()[:16]
+
+
+def ncu_traffic(workload: str):
+    """dram bytes per decode launch from the committed ncu summary, if it matches the
+    current kernel source; else None."""
+    f = ROOT / "profiles" / "decode_dram_traffic.json"
+    if not f.exists():
+        return None
+    d = json.loads(f.read_text())
+    entry = d.get(workload)
+    if not entry or entry.get("decode_source_sha") != decode_source_hash():
+        return None
+    return entry.get("dram_bytes_per_launch")
+
+
+class ClockSampler:
+    """nvidia-smi clock/throttle sampling during the timed region."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device: int):
+        self.gpu = str(device)
+        try:  # address the GPU by UUID so CUDA_VISIBLE_DEVICES remapping cannot mislead nvidia-smi
+            u = str(torch.cuda.get_device_properties(device).uuid)
+            self.gpu = u if u.startswith("GPU-") else "GPU-" + u
+        except Exception:
+            pass
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *exc):
+        self.lines = []
+        if self.proc is not None:
+            time.sleep(0.2)
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                out, _ = self.proc.communicate()
+            self.lines = [l for l in out.splitlines() if l.strip()]
+
+    def summary(self):
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for l in self.lines:
+            f = [x.strip() for x in l.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx.append(float(f[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        loaded = sorted(sm)[len(sm) // 4:] or sm  # drop the idle tail at the edges
+        return {"sm_mhz": statistics.median(loaded), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def time_oracle_sample(wl: synth.Workload, n_seqs: int, n_heads: int):
+    """Run the fp64 oracle (the expanded definition) on n_seqs x n_heads outputs of the
+    workload; return (seconds, (seq, head) pairs done, threads used)."""
+    import oracle
+    try:
+        import threadpoolctl
+        threads = max(i.get("num_threads", 1) for i in threadpoolctl.threadpool_info())
+    except Exception:  # pragma: no cover
+        threads = os.cpu_count()
+    w_uk, w_uv = synth.weights(wl)
+    q = synth.queries(wl)
+    lens = synth.seq_lens(wl)
+    seqs = list(range(min(n_seqs, wl.batch)))
+    heads = list(range(min(n_heads, wl.heads)))
+    rows = {s: synth.seq_rows(wl, s) for s in seqs}  # generation is not timed
+    t0 = time.perf_counter()
+    for s in seqs:
+        r = rows[s]
+        oracle.mlra_decode_expanded(q[s], r[:, :synth.D_C], r[:, synth.D_C:], w_uk, w_uv, wl.n_branch,
+                                    alpha_q=wl.alpha_q, alpha_kv=wl.alpha_kv, branch_scale=wl.sigma_o,
+                                    softmax_scale=wl.softmax_scale, rope_theta=wl.rope_theta, heads=heads)
+    dt = time.perf_counter() - t0
+    # the sample's share of the full step, by cached tokens x heads
+    frac = (sum(int(lens[s]) for s in seqs) * len(heads)) / (int(lens.sum()) * wl.heads)
+    return dt, frac, threads, len(seqs), len(heads)
+
+
+def workload_config(wl: synth.Workload, lens) -> dict:
+    return {"workload": wl.name, "variant": {1: "MLA", 2: "MLRA-2", 4: "MLRA-4"}[wl.n_branch],
+            "batch": wl.batch, "heads": wl.heads, "seq_len": wl.seq_len,
+            "seq_len_min": wl.seq_len_min, "total_tokens": int(np.asarray(lens, dtype=np.int64).sum()),
+            "layout": f"paged({wl.page_size})" if wl.page_size else "contiguous",
+            "d_c": 512, "d_rope": 64, "alpha_q": wl.alpha_q, "alpha_kv": wl.alpha_kv, "branch_scale": wl.sigma_o,
+            "l2": "inputs larger than L2 (KV cache per step >> 126 MB); no flush"}
+
+
+def dist_setup():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def run_reference(args, wl, world, rank):
+    if rank != 0:
+        return
+    lens = synth.seq_lens(wl)
+    kv = synth.kv_bytes(lens)
+    for _ in range(args.warmup):
+        time_oracle_sample(wl, 1, 1)
+    times = []
+    frac = threads = None
+    for _ in range(args.steps):
+        dt, frac, threads, ns, nh = time_oracle_sample(wl, args.ref_seqs, args.ref_heads)
+        times.append(dt / frac)  # extrapolated seconds per full decode step
+    step_s = statistics.mean(times)
+    value = kv / step_s / 1e12
+    sample = (f"each step: oracle (expanded fp64 definition) on {args.ref_seqs} sequence(s) x {args.ref_heads} "
+              f"head(s) of the workload, extrapolated by cached tokens x heads to the full step")
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "TB/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": step_s * 1e3,
+            "us_per_step": step_s * 1e6, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "f64", "data": "synthetic", "config": workload_config(wl, lens),
+            "cpu_baseline": {"value": value, "unit": "TB/s", "cores": threads, "kind": "oracle", "sample": sample},
+            "e2e": {"value": value, "unit": "TB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def run_native(args, wl, world, rank, local):
+    import head_rank_attention_b200 as hra
+    torch.cuda.set_device(local)
+    dev_id = torch.cuda.current_device()
+    if world > 1:
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+
+    inp = synth.make_inputs(wl)
+    lens = inp.seq_lens.numpy()
+    kv = synth.kv_bytes(lens)
+    dev = synth.to_device(inp)
+    stream = torch.cuda.current_stream()
+    out = torch.empty(wl.batch, wl.heads, synth.D_V, dtype=torch.float32, device="cuda")
+    p = hra.make_params(dev.q, dev.ckv, dev.krope, dev.seq_lens, dev.w_uk, dev.w_uv, out,
+                        n_branch=wl.n_branch, alpha_q=wl.alpha_q, alpha_kv=wl.alpha_kv, branch_scale=wl.sigma_o,
+                        softmax_scale=wl.softmax_scale, rope_theta=wl.rope_theta, block_table=dev.block_table,
+                        page_size=wl.page_size, seq_stride=dev.seq_stride, num_splits=args.num_splits)
+    ws = hra.alloc_workspace(p)
+
+    # per-step stage events: [before absorb, before decode, before combine, after combine]
+    events = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    handles = [(ctypes.c_void_p * 4)(*[e.cuda_event for e in evs]) for evs in events]
+
+    for _ in range(args.warmup):
+        hra.mlra_decode(p, stream)
+    hra.check_device_status(p, stream)
+
+    def barrier():
+        if world > 1:
+            torch.distributed.barrier()
+        torch.cuda.synchronize()
+
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    with ClockSampler(dev_id) as clk:
+        start.record(stream)
+        for k in range(args.steps):
+            p.stage_events = ctypes.cast(handles[k], ctypes.c_void_p)
+            hra.mlra_decode(p, stream)
+        end.record(stream)
+        torch.cuda.synchronize()
+    p.stage_events = None
+    hra.check_device_status(p, stream)
+    elapsed_ms = start.elapsed_time(end)
+    stage_ms = np.array([[evs[i].elapsed_time(evs[i + 1]) for i in range(3)] for evs in events])
+    decode_ms = float(stage_ms[:, 1].mean())
+
+    # end to end through the C ABI with host buffers: H2D of every input, decode, D2H of out
+    pin = {k: v.pin_memory() for k, v in dict(q=inp.q, cache=inp.cache, seq_lens=inp.seq_lens,
+                                               w_uk=inp.w_uk, w_uv=inp.w_uv).items()}
+    if inp.block_table is not None:
+        pin["block_table"] = inp.block_table.pin_memory()
+    host_out = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
+    dmap = dict(q=dev.q, cache=dev.cache, seq_lens=dev.seq_lens, w_uk=dev.w_uk, w_uv=dev.w_uv,
+                block_table=dev.block_table)
+    h2d = sum(t.numel() * t.element_size() for t in pin.values())
+    d2h = host_out.numel() * host_out.element_size()
+    e2e_steps = max(1, min(args.steps, args.e2e_steps))
+    barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        for k, t in pin.items():
+            dmap[k].copy_(t, non_blocking=True)
+        hra.mlra_decode(p, stream)
+        host_out.copy_(out, non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1) / e2e_steps
+    hra.check_device_status(p, stream)
+
+    step_ms = elapsed_ms / args.steps
+    if world > 1:
+        t = torch.tensor([step_ms, e2e_ms, decode_ms], device="cuda", dtype=torch.float64)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        step_ms, e2e_ms, decode_ms = (float(x) for x in t.cpu())
+    clocks = clk.summary()
+
+    if rank == 0:
+        pk, pk_src = peaks()
+        achieved_gbs = kv / (decode_ms * 1e-3) / 1e9
+        flops = tensor_flops_per_token(wl.n_branch, wl.heads) * int(lens.astype(np.int64).sum())
+        achieved_tflops = flops / (decode_ms * 1e-3) / 1e12
+        traffic = ncu_traffic(wl.name)
+        line = {
+            "metric": METRIC,
+            "value": world * kv / (step_ms * 1e-3) / 1e12, "unit": "TB/s",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": step_ms, "us_per_step": step_ms * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "f16", "precision": "bf16 inputs; fp16 tensor-core operands; fp32 accumulate, softmax, combine",
+            "data": "synthetic",
+            "config": dict(workload_config(wl, lens), parallelism=f"replicas x{world}" if world > 1 else "1 GPU",
+                           num_splits=args.num_splits or "auto (SMs/4)"),
+            "kv_frac_of_nominal_8TBs": kv / (step_ms * 1e-3) / 1e9 / NOMINAL_HBM_GBS,
+            "stage_us": {"absorb_q": float(stage_ms[:, 0].mean()) * 1e3, "decode": decode_ms * 1e3,
+                         "combine_upproj": float(stage_ms[:, 2].mean()) * 1e3},
+            "roofline": {"kernel": "decode_kernel (split-KV tcgen05)", "bound": "hbm", "achieved": achieved_gbs,
+                         "peak": pk["hbm_gbs"], "unit": "GB/s", "frac": achieved_gbs / pk["hbm_gbs"],
+                         "peak_source": pk_src, "traffic": traffic,
+                         "bytes_per_launch": kv},
+            "roofline_tensor": {"achieved": achieved_tflops, "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
+                                "frac": achieved_tflops / pk["bf16_tflops"],
+                                "note": "fp16 operands, same dense peak as bf16; algorithmic FLOPs"},
+            "clocks": clocks,
+            "e2e": {"value": world * kv / (e2e_ms * 1e-3) / 1e12, "unit": "TB/s", "ms_per_step": e2e_ms,
+                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": e2e_steps},
+            "gpu_launches": 3 * args.steps,
+        }
+        if world == 1 and not args.no_cpu_baseline:
+            dt, frac, threads, ns, nh = time_oracle_sample(wl, args.cpu_seqs, args.cpu_heads)
+            cpu_step = dt / frac
+            line["cpu_baseline"] = {
+                "value": kv / cpu_step / 1e12, "unit": "TB/s", "cores": threads, "kind": "oracle",
+                "us_per_step": cpu_step * 1e6, "seconds_measured": dt,
+                "sample": (f"fp64 expanded-definition oracle on {ns} sequence(s) x {nh} head(s), "
+                           f"extrapolated by cached tokens x heads to the full step")}
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        torch.distributed.barrier()
+        torch.distributed.destroy_process_group()
+    del ws
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["native", "reference"], default="native")
+    ap.add_argument("--workload", default="paged_b64_t32k_mlra4", choices=sorted(synth.WORKLOADS))
+    ap.add_argument("--num-splits", type=int, default=0)
+    ap.add_argument("--e2e-steps", type=int, default=5)
+    ap.add_argument("--cpu-seqs", type=int, default=4)
+    ap.add_argument("--cpu-heads", type=int, default=16)
+    ap.add_argument("--ref-seqs", type=int, default=1)
+    ap.add_argument("--ref-heads", type=int, default=8)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    world, rank, local = dist_setup()
+    wl = synth.WORKLOADS[args.workload]
+    if args.impl == "reference":
+        run_reference(args, wl, world, rank)
+    else:
+        run_native(args, wl, world, rank, local)
+
+
+if __name__ == "__main__":
+    main()

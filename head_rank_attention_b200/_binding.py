@@ -1,0 +1,174 @@
+"""ctypes binding of libhra.so (include/hra.h).  Argument marshalling only: every step of
+the decode runs in the library's CUDA kernels.  There is no fallback: if the library is
+missing or fails to load, importing a call raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import pathlib
+from typing import Optional
+
+LIB_PATH = pathlib.Path(__file__).resolve().with_name("libhra.so")
+
+HRA_OK = 0
+HRA_ERR_INVALID_ARG = -1
+HRA_ERR_UNSUPPORTED = -2
+HRA_ERR_WORKSPACE = -3
+HRA_ERR_CUDA = -4
+HRA_ERR_DEVICE_TIMEOUT = -5
+HRA_BF16 = 0
+HRA_F32 = 1
+
+STATUS_NAMES = {0: "HRA_OK", -1: "HRA_ERR_INVALID_ARG", -2: "HRA_ERR_UNSUPPORTED", -3: "HRA_ERR_WORKSPACE",
+                -4: "HRA_ERR_CUDA", -5: "HRA_ERR_DEVICE_TIMEOUT"}
+
+# Symbols declared in include/hra.h.
+EXPORTS = ("hra_workspace_size", "mlra_decode", "mla_decode", "hra_check_device_status",
+           "hra_selftest_wait_timeout", "hra_last_error", "hra_version")
+
+
+class HraError(RuntimeError):
+    def __init__(self, status: int, message: str):
+        super().__init__(f"{STATUS_NAMES.get(status, status)}: {message}")
+        self.status = status
+
+
+class HraDecodeParams(ctypes.Structure):
+    """Mirror of hra_decode_params (field order and C types as in include/hra.h)."""
+    _fields_ = [
+        ("batch", ctypes.c_int), ("num_heads", ctypes.c_int), ("n_branch", ctypes.c_int),
+        ("d_c", ctypes.c_int), ("d_rope", ctypes.c_int), ("d_nope", ctypes.c_int), ("d_v", ctypes.c_int),
+        ("q", ctypes.c_void_p), ("ckv", ctypes.c_void_p), ("krope", ctypes.c_void_p),
+        ("ckv_stride", ctypes.c_int64), ("krope_stride", ctypes.c_int64), ("cache_rows", ctypes.c_int64),
+        ("seq_lens", ctypes.c_void_p), ("block_table", ctypes.c_void_p),
+        ("max_pages", ctypes.c_int32), ("page_size", ctypes.c_int32), ("seq_stride", ctypes.c_int64),
+        ("w_uk", ctypes.c_void_p), ("w_uv", ctypes.c_void_p),
+        ("alpha_q", ctypes.c_float), ("alpha_kv", ctypes.c_float), ("branch_scale", ctypes.c_float),
+        ("softmax_scale", ctypes.c_float), ("rope_theta", ctypes.c_float),
+        ("out", ctypes.c_void_p), ("out_dtype", ctypes.c_int),
+        ("workspace", ctypes.c_void_p), ("workspace_bytes", ctypes.c_size_t),
+        ("num_splits", ctypes.c_int), ("wait_limit", ctypes.c_int),
+        ("stage_events", ctypes.c_void_p),
+    ]
+
+
+_lib: Optional[ctypes.CDLL] = None
+
+
+def load_library() -> ctypes.CDLL:
+    """Load libhra.so from the package directory (raises if it is not built)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not LIB_PATH.exists():
+        raise ImportError(f"{LIB_PATH} is not built; run `python -m head_rank_attention_b200.build`")
+    lib = ctypes.CDLL(str(LIB_PATH))
+    P = ctypes.POINTER(HraDecodeParams)
+    lib.hra_workspace_size.argtypes = [P]
+    lib.hra_workspace_size.restype = ctypes.c_size_t
+    for name in ("mlra_decode", "mla_decode", "hra_check_device_status"):
+        getattr(lib, name).argtypes = [P, ctypes.c_void_p]
+        getattr(lib, name).restype = ctypes.c_int
+    lib.hra_selftest_wait_timeout.argtypes = [ctypes.c_void_p, ctypes.c_int, ctypes.c_void_p]
+    lib.hra_selftest_wait_timeout.restype = ctypes.c_int
+    lib.hra_last_error.argtypes = []
+    lib.hra_last_error.restype = ctypes.c_char_p
+    lib.hra_version.argtypes = []
+    lib.hra_version.restype = ctypes.c_char_p
+    _lib = lib
+    return lib
+
+
+def last_error() -> str:
+    return load_library().hra_last_error().decode()
+
+
+def version() -> str:
+    return load_library().hra_version().decode()
+
+
+def _check(status: int) -> None:
+    if status != HRA_OK:
+        raise HraError(status, last_error())
+
+
+def _stream_handle(stream) -> int:
+    if stream is None:
+        import torch
+        return torch.cuda.current_stream().cuda_stream
+    return getattr(stream, "cuda_stream", stream)
+
+
+def _ptr(t) -> int:
+    return 0 if t is None else int(t.data_ptr())
+
+
+def make_params(q, ckv, krope, seq_lens, w_uk, w_uv, out, workspace=None, *, n_branch: int,
+                alpha_q: float = 1.0, alpha_kv: float = 1.0, branch_scale: Optional[float] = None,
+                softmax_scale: float = 0.0, rope_theta: float = 10000.0, block_table=None,
+                page_size: int = 0, seq_stride: int = 0, cache_rows: Optional[int] = None,
+                num_splits: int = 0, wait_limit: int = 0) -> HraDecodeParams:
+    """Fill hra_decode_params from torch tensors (shapes/dtypes as documented in hra.h).
+
+    ckv / krope are 2-D row views of the cache (e.g. cache[:, :512], cache[:, 512:]);
+    their row strides become ckv_stride / krope_stride.
+    """
+    import torch
+    p = HraDecodeParams()
+    p.batch, p.num_heads = int(q.shape[0]), int(q.shape[1])
+    p.n_branch = int(n_branch)
+    p.d_c, p.d_rope, p.d_nope, p.d_v = int(ckv.shape[1]), int(krope.shape[1]), int(q.shape[2]) - int(krope.shape[1]), int(w_uv.shape[2])
+    p.q, p.ckv, p.krope = _ptr(q), _ptr(ckv), _ptr(krope)
+    p.ckv_stride, p.krope_stride = int(ckv.stride(0)), int(krope.stride(0))
+    p.cache_rows = int(ckv.shape[0]) if cache_rows is None else int(cache_rows)
+    p.seq_lens = _ptr(seq_lens)
+    p.block_table = _ptr(block_table)
+    p.max_pages = int(block_table.shape[1]) if block_table is not None else 0
+    p.page_size = int(page_size)
+    p.seq_stride = int(seq_stride)
+    p.w_uk, p.w_uv = _ptr(w_uk), _ptr(w_uv)
+    p.alpha_q, p.alpha_kv = float(alpha_q), float(alpha_kv)
+    p.branch_scale = float(1.0 / math.sqrt(n_branch) if branch_scale is None else branch_scale)
+    p.softmax_scale, p.rope_theta = float(softmax_scale), float(rope_theta)
+    p.out = _ptr(out)
+    p.out_dtype = HRA_F32 if out is not None and out.dtype == torch.float32 else HRA_BF16
+    p.workspace = _ptr(workspace)
+    p.workspace_bytes = 0 if workspace is None else int(workspace.numel() * workspace.element_size())
+    p.num_splits, p.wait_limit = int(num_splits), int(wait_limit)
+    return p
+
+
+def workspace_size(p: HraDecodeParams) -> int:
+    n = load_library().hra_workspace_size(ctypes.byref(p))
+    if n == 0:
+        raise HraError(HRA_ERR_INVALID_ARG, last_error())
+    return int(n)
+
+
+def mlra_decode(p: HraDecodeParams, stream=None) -> None:
+    _check(load_library().mlra_decode(ctypes.byref(p), ctypes.c_void_p(_stream_handle(stream))))
+
+
+def mla_decode(p: HraDecodeParams, stream=None) -> None:
+    _check(load_library().mla_decode(ctypes.byref(p), ctypes.c_void_p(_stream_handle(stream))))
+
+
+def check_device_status(p: HraDecodeParams, stream=None) -> None:
+    _check(load_library().hra_check_device_status(ctypes.byref(p), ctypes.c_void_p(_stream_handle(stream))))
+
+
+def selftest_wait_timeout(workspace, limit_us: int, stream=None) -> None:
+    _check(load_library().hra_selftest_wait_timeout(ctypes.c_void_p(_ptr(workspace)), int(limit_us),
+                                                    ctypes.c_void_p(_stream_handle(stream))))
+
+
+def alloc_workspace(p: HraDecodeParams, device=None):
+    """Allocate a workspace for p with torch (256-byte aligned) and attach it to p."""
+    import torch
+    n = workspace_size(p)
+    ws = torch.empty(n + 256, dtype=torch.uint8, device=device or "cuda")
+    off = (-ws.data_ptr()) % 256
+    ws = ws[off:off + n]
+    p.workspace, p.workspace_bytes = ws.data_ptr(), n
+    return ws

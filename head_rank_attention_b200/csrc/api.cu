@@ -1,0 +1,298 @@
+// api.cu -- the C ABI of libhra.so (declared in include/hra.h): argument validation,
+// workspace layout, TMA descriptor encoding and the launch sequence
+//   absorb_q  ->  decode (split-KV, tcgen05)  ->  combine_upproj
+// of one decode step, all on the caller's stream.  Nothing here allocates device memory.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+#include <string>
+
+#include "hra.h"
+#include "absorb_combine.h"
+#include "decode_sm100.h"
+#include "schedule.cuh"
+#include "sm100.cuh"
+
+namespace {
+
+thread_local std::string g_last_error;
+
+hra_status fail(hra_status st, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  g_last_error = buf;
+  return st;
+}
+
+hra_status cuda_fail(cudaError_t e, const char* what) {
+  return fail(HRA_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+constexpr uint64_t kDefaultWaitLimitUs = 1000000;  // 1 s per device-side wait
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+size_t round256(size_t x) { return (x + 255) & ~size_t(255); }
+
+struct Plan {
+  int groups = 0;
+  long long slots = 0;
+  size_t q_tilde = 0, o_part = 0, ml_part = 0, total = 0;
+};
+
+hra_status sm_count(int* n) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  e = cudaDeviceGetAttribute(n, cudaDevAttrMultiProcessorCount, dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceGetAttribute");
+  return HRA_OK;
+}
+
+hra_status validate(const hra_decode_params* p) {
+  if (p == nullptr) return fail(HRA_ERR_INVALID_ARG, "params is NULL");
+  if (p->d_c != 512 || p->d_rope != 64 || p->d_nope != 128 || p->d_v != 128)
+    return fail(HRA_ERR_UNSUPPORTED, "widths (d_c=%d, d_rope=%d, d_nope=%d, d_v=%d) must be 512/64/128/128",
+                p->d_c, p->d_rope, p->d_nope, p->d_v);
+  if (p->n_branch != 1 && p->n_branch != 2 && p->n_branch != 4)
+    return fail(HRA_ERR_UNSUPPORTED, "n_branch=%d (supported: 1, 2, 4)", p->n_branch);
+  if (p->batch < 1 || p->batch > hra::kMaxBatch)
+    return fail(HRA_ERR_UNSUPPORTED, "batch=%d (supported: 1..%d)", p->batch, hra::kMaxBatch);
+  if (p->num_heads < 1 || p->num_heads > 128)
+    return fail(HRA_ERR_UNSUPPORTED, "num_heads=%d (supported: 1..128)", p->num_heads);
+  const struct { const void* ptr; const char* name; } ptrs[] = {
+      {p->q, "q"}, {p->ckv, "ckv"}, {p->krope, "krope"}, {p->seq_lens, "seq_lens"},
+      {p->w_uk, "w_uk"}, {p->w_uv, "w_uv"}, {p->out, "out"}};
+  for (const auto& x : ptrs) {
+    if (x.ptr == nullptr) return fail(HRA_ERR_INVALID_ARG, "%s is NULL", x.name);
+    if (!aligned16(x.ptr)) return fail(HRA_ERR_INVALID_ARG, "%s is not 16-byte aligned", x.name);
+  }
+  if (p->ckv_stride < 512 || p->ckv_stride % 8 != 0)
+    return fail(HRA_ERR_INVALID_ARG, "ckv_stride=%lld must be >= 512 and a multiple of 8", (long long)p->ckv_stride);
+  if (p->krope_stride < 64 || p->krope_stride % 8 != 0)
+    return fail(HRA_ERR_INVALID_ARG, "krope_stride=%lld must be >= 64 and a multiple of 8",
+                (long long)p->krope_stride);
+  if (p->cache_rows < 1 || p->cache_rows > 0x7FFFFFFFLL)
+    return fail(HRA_ERR_INVALID_ARG, "cache_rows=%lld out of range [1, 2^31-1]", (long long)p->cache_rows);
+  if (p->block_table != nullptr) {
+    if (p->max_pages < 1) return fail(HRA_ERR_INVALID_ARG, "max_pages=%d must be >= 1", p->max_pages);
+    if (p->page_size < 32 || p->page_size % 32 != 0)
+      return fail(HRA_ERR_UNSUPPORTED, "page_size=%d must be a positive multiple of 32", p->page_size);
+  } else if (p->seq_stride < 0) {
+    return fail(HRA_ERR_INVALID_ARG, "seq_stride=%lld must be >= 0", (long long)p->seq_stride);
+  }
+  if (p->out_dtype != HRA_BF16 && p->out_dtype != HRA_F32)
+    return fail(HRA_ERR_INVALID_ARG, "out_dtype=%d", (int)p->out_dtype);
+  if (p->num_splits < 0) return fail(HRA_ERR_INVALID_ARG, "num_splits=%d must be >= 0", p->num_splits);
+  if (p->wait_limit < 0) return fail(HRA_ERR_INVALID_ARG, "wait_limit=%d must be >= 0", p->wait_limit);
+  if (!std::isfinite(p->alpha_q) || !std::isfinite(p->alpha_kv) || !std::isfinite(p->branch_scale) ||
+      !std::isfinite(p->softmax_scale) || !(p->rope_theta > 0.f) || !std::isfinite(p->rope_theta))
+    return fail(HRA_ERR_INVALID_ARG, "scales must be finite and rope_theta > 0");
+  return HRA_OK;
+}
+
+hra_status make_plan(const hra_decode_params* p, Plan* plan) {
+  int sms = 0;
+  if (p->num_splits > 0) {
+    plan->groups = p->num_splits;
+  } else {
+    hra_status st = sm_count(&sms);
+    if (st != HRA_OK) return st;
+    plan->groups = sms / 4 > 0 ? sms / 4 : 1;
+  }
+  if (plan->groups > 65535) return fail(HRA_ERR_INVALID_ARG, "num_splits=%d too large", plan->groups);
+  plan->slots = static_cast<long long>(plan->groups) + p->batch;
+  size_t off = 256;  // device status word
+  plan->q_tilde = off;
+  off = round256(off + static_cast<size_t>(p->batch) * p->num_heads * 576 * sizeof(__half));
+  plan->o_part = off;
+  off = round256(off + static_cast<size_t>(plan->slots) * 4 * 128 * 128 * sizeof(float));
+  plan->ml_part = off;
+  off = round256(off + static_cast<size_t>(plan->slots) * 4 * 128 * sizeof(float2));
+  plan->total = off;
+  return HRA_OK;
+}
+
+std::once_flag g_encode_once;
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+
+hra_status encode_map(CUtensorMap* map, const void* base, int64_t inner, int64_t rows, int64_t stride_elems) {
+  std::call_once(g_encode_once, [] {
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q{};
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+  });
+  if (g_encode == nullptr) return fail(HRA_ERR_CUDA, "cuTensorMapEncodeTiled entry point unavailable");
+  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(inner), static_cast<cuuint64_t>(rows)};
+  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(stride_elems) * 2};
+  const cuuint32_t box[2] = {64, 32};
+  const cuuint32_t estr[2] = {1, 1};
+  CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(HRA_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
+  return HRA_OK;
+}
+
+hra_status run_decode(const hra_decode_params* p, cudaStream_t stream) {
+  hra_status st = validate(p);
+  if (st != HRA_OK) return st;
+  Plan plan;
+  st = make_plan(p, &plan);
+  if (st != HRA_OK) return st;
+  if (p->workspace == nullptr) return fail(HRA_ERR_WORKSPACE, "workspace is NULL");
+  if ((reinterpret_cast<uintptr_t>(p->workspace) & 255u) != 0)
+    return fail(HRA_ERR_WORKSPACE, "workspace is not 256-byte aligned");
+  if (p->workspace_bytes < plan.total)
+    return fail(HRA_ERR_WORKSPACE, "workspace_bytes=%zu < required %zu", p->workspace_bytes, plan.total);
+
+  uint8_t* ws = static_cast<uint8_t*>(p->workspace);
+  int* status = reinterpret_cast<int*>(ws);
+  __half* q_tilde = reinterpret_cast<__half*>(ws + plan.q_tilde);
+  float* o_part = reinterpret_cast<float*>(ws + plan.o_part);
+  float2* ml_part = reinterpret_cast<float2*>(ws + plan.ml_part);
+
+  auto mark = [&](int k) -> cudaError_t {
+    return p->stage_events ? cudaEventRecord(static_cast<cudaEvent_t>(p->stage_events[k]), stream) : cudaSuccess;
+  };
+  cudaError_t e = mark(0);
+  if (e != cudaSuccess) return cuda_fail(e, "stage event");
+
+  hra::AbsorbArgs ab{};
+  ab.q = static_cast<const __nv_bfloat16*>(p->q);
+  ab.w_uk = static_cast<const __nv_bfloat16*>(p->w_uk);
+  ab.seq_lens = p->seq_lens;
+  ab.q_tilde = q_tilde;
+  ab.status = status;
+  ab.batch = p->batch;
+  ab.heads = p->num_heads;
+  ab.alpha_q = p->alpha_q;
+  ab.alpha_kv = p->alpha_kv;
+  ab.rope_theta = p->rope_theta;
+  e = hra::launch_absorb_q(ab, stream);
+  if (e != cudaSuccess) return cuda_fail(e, "absorb_q launch");
+
+  CUtensorMap map_ckv, map_krope;
+  st = encode_map(&map_ckv, p->ckv, 512, p->cache_rows, p->ckv_stride);
+  if (st != HRA_OK) return st;
+  st = encode_map(&map_krope, p->krope, 64, p->cache_rows, p->krope_stride);
+  if (st != HRA_OK) return st;
+
+  const float tau = p->softmax_scale > 0.f ? p->softmax_scale : 1.0f / std::sqrt(192.0f);
+  hra::DecodeArgs da{};
+  da.q_tilde = q_tilde;
+  da.seq_lens = p->seq_lens;
+  da.block_table = p->block_table;
+  da.max_pages = p->max_pages;
+  da.page_size = p->page_size;
+  da.seq_stride = p->seq_stride;
+  da.cache_rows = p->cache_rows;
+  da.batch = p->batch;
+  da.heads = p->num_heads;
+  da.scale_log2 = tau * 1.4426950408889634f;
+  da.o_part = o_part;
+  da.ml_part = ml_part;
+  da.status = status;
+  da.wait_limit_ns = 1000ull * (p->wait_limit > 0 ? static_cast<uint64_t>(p->wait_limit) : kDefaultWaitLimitUs);
+  if ((e = mark(1)) != cudaSuccess) return cuda_fail(e, "stage event");
+  e = hra::launch_decode_kernel(p->n_branch, map_ckv, map_krope, da, plan.groups, stream);
+  if (e != cudaSuccess) return cuda_fail(e, "decode launch");
+  if ((e = mark(2)) != cudaSuccess) return cuda_fail(e, "stage event");
+
+  hra::CombineArgs cb{};
+  cb.o_part = o_part;
+  cb.ml_part = ml_part;
+  cb.seq_lens = p->seq_lens;
+  cb.w_uv = static_cast<const __nv_bfloat16*>(p->w_uv);
+  cb.out_f32 = p->out_dtype == HRA_F32 ? static_cast<float*>(p->out) : nullptr;
+  cb.out_bf16 = p->out_dtype == HRA_BF16 ? static_cast<__nv_bfloat16*>(p->out) : nullptr;
+  cb.batch = p->batch;
+  cb.heads = p->num_heads;
+  cb.groups = plan.groups;
+  cb.tile_tokens = hra::decode_tile_tokens(p->n_branch);
+  cb.alpha_kv = p->alpha_kv;
+  cb.branch_scale = p->branch_scale;
+  e = hra::launch_combine_upproj(cb, stream);
+  if (e != cudaSuccess) return cuda_fail(e, "combine_upproj launch");
+  if ((e = mark(3)) != cudaSuccess) return cuda_fail(e, "stage event");
+  g_last_error.clear();
+  return HRA_OK;
+}
+
+__global__ void wait_timeout_selftest_kernel(int* status, uint64_t limit_ns) {
+  __shared__ uint64_t bar;
+  __shared__ volatile int abort_flag;
+  if (threadIdx.x == 0) {
+    status[0] = status[1] = status[2] = status[3] = 0;
+    hra::mbar_init(&bar, 1);
+    abort_flag = 0;
+    hra::fence_mbar_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    // nothing ever arrives on `bar`: the wait must give up after limit_ns
+    hra::mbar_wait(&bar, 0, limit_ns, &abort_flag, status, 99);
+  }
+  __syncthreads();
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t hra_workspace_size(const hra_decode_params* p) {
+  if (validate(p) != HRA_OK) return 0;
+  Plan plan;
+  if (make_plan(p, &plan) != HRA_OK) return 0;
+  return plan.total;
+}
+
+hra_status mlra_decode(const hra_decode_params* p, void* stream) {
+  return run_decode(p, static_cast<cudaStream_t>(stream));
+}
+
+hra_status mla_decode(const hra_decode_params* p, void* stream) {
+  if (p != nullptr && p->n_branch != 1)
+    return fail(HRA_ERR_INVALID_ARG, "mla_decode requires n_branch == 1 (got %d)", p->n_branch);
+  return run_decode(p, static_cast<cudaStream_t>(stream));
+}
+
+hra_status hra_check_device_status(const hra_decode_params* p, void* stream) {
+  if (p == nullptr || p->workspace == nullptr) return fail(HRA_ERR_INVALID_ARG, "params or workspace is NULL");
+  cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");
+  int st[4] = {0, 0, 0, 0};
+  e = cudaMemcpy(st, p->workspace, sizeof(st), cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return cuda_fail(e, "status read");
+  if (st[0] != 0)
+    return fail(HRA_ERR_DEVICE_TIMEOUT, "device wait expired (code %d, site %d, parity %d, block %d)", st[0], st[1],
+                st[2], st[3]);
+  g_last_error.clear();
+  return HRA_OK;
+}
+
+hra_status hra_selftest_wait_timeout(void* workspace, int limit_us, void* stream) {
+  if (workspace == nullptr) return fail(HRA_ERR_INVALID_ARG, "workspace is NULL");
+  if (limit_us < 1 || limit_us > 10000000) return fail(HRA_ERR_INVALID_ARG, "limit_us=%d out of [1, 1e7]", limit_us);
+  wait_timeout_selftest_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(
+      static_cast<int*>(workspace), 1000ull * static_cast<uint64_t>(limit_us));
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "selftest launch");
+  return HRA_OK;
+}
+
+const char* hra_last_error(void) { return g_last_error.c_str(); }
+
+const char* hra_version(void) { return "hra 0.1.0 (sm_100a)"; }
+
+}  // extern "C"

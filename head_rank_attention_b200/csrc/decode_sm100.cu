@@ -1,0 +1,463 @@
+// decode_sm100.cu -- split-KV latent-cache decode on tcgen05/TMEM with TMA tile streams.
+//
+// Step 2 of the decode in "Multi-Head Low-Rank Attention" (方法步骤详情): MQA-style
+// attention of the absorbed per-head queries over the shared key [C_KV | K_RoPE] and
+// value C_KV, one independent softmax per (head, branch) (核心方法:
+// O = sum_b Softmax(Q K_b^T) V_b; MLA is the single-branch case).
+//
+// Work decomposition (one CTA per SM):
+//   blockIdx.x = slice c in 0..3: the CTA owns output latent columns [128c, 128c+128),
+//                which belong to branch b = c / (W/128) of width W = 512/NB;
+//   blockIdx.y = group g: a contiguous range of cache tiles (see schedule.cuh).
+// A CTA streams, for every tile of NT tokens, the branch's W latent columns plus the 64
+// RoPE columns (TMA, 64x32 boxes, 128-byte swizzle), converts them to fp16 in shared
+// memory, computes S = Q~_b [C_b | K_R]^T for all 128 head rows with tcgen05 (A = Q~
+// from TMEM, B = the tile, D = S in TMEM), runs the online softmax with one thread per
+// head row, writes P (fp16) back over S in TMEM and accumulates O += P V with V = its
+// 128 latent columns of the same tile (A = P from TMEM, B = MN-major tile).  Each
+// segment ends by writing the un-normalised O row, the running max m (log2 units) and
+// the row sum l of every head to the workspace.
+//
+// Warp roles: warps 0-3 softmax + epilogue (thread = head row = TMEM lane), warps 4-7
+// bf16 -> fp16 conversion, warp 8 TMA producer, warp 9 TMEM allocator + MMA issuer.
+// Every wait is bounded (see sm100.cuh); on expiry the CTA drains and exits with the
+// failure recorded in the workspace status word.
+
+#include <cstdint>
+
+#include "decode_sm100.h"
+#include "schedule.cuh"
+#include "sm100.cuh"
+
+namespace hra {
+
+template <int NB, int NT, int STAGES>
+struct DecodeCfg {
+  static constexpr int NT_ = NT;
+  static constexpr int STAGES_ = STAGES;
+  static constexpr int W = 512 / NB;                 // branch width
+  static constexpr int QK_DIMS = W + 64;             // contraction length of one score
+  static constexpr int QK_BOXES = QK_DIMS / 64;      // 64-wide boxes per tile (last = rope)
+  static constexpr int SLICES_PER_BRANCH = W / 128;
+  static constexpr int BOX_BYTES = NT * 128;         // one 64-column box over NT rows
+  static constexpr int STAGE_BYTES = QK_BOXES * BOX_BYTES;
+  static constexpr int CHUNKS = NT / 32;             // TMA row chunks per tile
+  static constexpr int TMEM_O = 0;                   // O: 128 fp32 columns
+  static constexpr int TMEM_S = 128;                 // S/P double buffer: 2 x NT columns
+  static constexpr int TMEM_Q = 128 + 2 * NT;        // Q~ (fp16 pairs): QK_DIMS/2 columns
+  static constexpr int TMEM_COLS = 512;
+  static constexpr int THREADS = 320;
+  static constexpr int MISC_BYTES = 256 + 4 * (kMaxBatch + 1);
+  static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + MISC_BYTES;
+  static_assert(TMEM_Q + QK_DIMS / 2 <= TMEM_COLS, "TMEM budget");
+  static_assert(NT % 32 == 0 && NT >= 32 && NT <= 256, "tile rows");
+  static_assert(SMEM_BYTES <= 232448, "shared memory budget");
+};
+
+namespace {
+
+// All lanes of a warp poll; the result is made warp-uniform so that the .sync.aligned
+// tcgen05 instructions and warp votes that follow see a converged warp.
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, uint64_t limit, volatile int* abort,
+                                          int* status, int where) {
+  const bool ok = mbar_wait(bar, parity, limit, abort, status, where);
+  return __all_sync(0xffffffffu, ok);
+}
+
+// Smallest sequence index s with prefix[s + 1] > t.
+__device__ __forceinline__ int first_seq(const int* prefix, int B, int t) {
+  int lo = 0, hi = B - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi) >> 1;
+    if (prefix[mid + 1] > t) hi = mid; else lo = mid + 1;
+  }
+  return lo;
+}
+
+// O += P V for cache tile number `tile_it` (CTA-local count): A = P (fp16) from the S/P
+// buffer the tile used, B = this slice's 128 latent columns of the tile (MN-major).
+template <class C>
+__device__ __forceinline__ void issue_pv(uint32_t tiles_addr, uint32_t tmem, uint64_t* pv_done, uint64_t* empty,
+                                         int tile_it, bool first, int pv_box) {
+  constexpr int NT = C::NT_;
+  constexpr uint32_t idesc_pv = idesc_f16_f32(128, 128, true);
+  const int stage = tile_it % C::STAGES_;
+  const uint32_t sb = tile_it & 1;
+  const uint32_t v_base = tiles_addr + stage * C::STAGE_BYTES + pv_box * C::BOX_BYTES;
+#pragma unroll
+  for (int k = 0; k < NT / 16; ++k) {
+    const uint64_t bdesc = smem_desc_sw128(v_base + k * 16 * 128, C::BOX_BYTES, 1024);
+    umma_f16_ts(tmem + C::TMEM_O, tmem + C::TMEM_S + sb * NT + k * 8, bdesc, idesc_pv,
+                (first && k == 0) ? 0u : 1u);
+  }
+  umma_commit(pv_done);
+  umma_commit(&empty[stage]);
+}
+
+template <int NB, int NT, int STAGES>
+__global__ void __launch_bounds__(320, 1)
+decode_kernel(const __grid_constant__ CUtensorMap map_ckv, const __grid_constant__ CUtensorMap map_krope,
+              const DecodeArgs a) {
+  using C = DecodeCfg<NB, NT, STAGES>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* tiles = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(tiles + STAGES * C::STAGE_BYTES);
+  uint64_t* conv = full + STAGES;
+  uint64_t* empty = conv + STAGES;
+  uint64_t* s_full = empty + STAGES;  // [2]
+  uint64_t* p_ready = s_full + 2;     // [2]
+  uint64_t* pv_done = p_ready + 2;
+  uint64_t* q_ready = pv_done + 1;
+  uint64_t* drain = q_ready + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  int* prefix = reinterpret_cast<int*>(tiles + STAGES * C::STAGE_BYTES + 256);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int slice = blockIdx.x;
+  const int branch = slice / C::SLICES_PER_BRANCH;
+  const int pv_box = (slice % C::SLICES_PER_BRANCH) * 2;  // first of the 2 boxes holding V
+  const int G = gridDim.y;
+  const int g = blockIdx.y;
+  const int B = a.batch;
+  const uint64_t limit = a.wait_limit_ns;
+  int* status = a.status;
+
+  if (warp == 0) tile_prefix_warp(a.seq_lens, B, NT, prefix);
+  if (threadIdx.x == 32) {
+    for (int i = 0; i < STAGES; ++i) {
+      mbar_init(&full[i], 1);
+      mbar_init(&conv[i], 128);
+      mbar_init(&empty[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&s_full[i], 1);
+      mbar_init(&p_ready[i], 128);
+    }
+    mbar_init(pv_done, 1);
+    mbar_init(q_ready, 128);
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 9) {
+    tmem_alloc(tmem_slot, C::TMEM_COLS);
+    tmem_relinquish();
+  }
+  if (warp == 8 && lane == 0) {
+    tma_prefetch_desc(&map_ckv);
+    tma_prefetch_desc(&map_krope);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  const int T = prefix[B];
+  const int t_begin = T > 0 ? group_tile_begin(g, G, T) : 0;
+  const int t_end = T > 0 ? group_tile_begin(g + 1, G, T) : 0;
+  const int s_first = (t_begin < t_end) ? first_seq(prefix, B, t_begin) : B;
+
+  if (warp == 8) {
+    // ------------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      const uint64_t policy = l2_policy_evict_first();
+      int it = 0;
+      bool ok = true;
+      for (int s = s_first; ok && s < B && prefix[s] < t_end; ++s) {
+        const int j0 = max(t_begin, prefix[s]), j1 = min(t_end, prefix[s + 1]);
+        if (j0 >= j1) continue;  // empty sequence: no tiles, no segment
+        const int L = a.seq_lens[s];
+        for (int j = j0; j < j1; ++j, ++it) {
+          const int stage = it % STAGES;
+          if (it >= STAGES &&
+              !mbar_wait(&empty[stage], ((it / STAGES) + 1) & 1, limit, abort_flag, status, 1)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(&full[stage], C::STAGE_BYTES);
+          const int tok0 = (j - prefix[s]) * NT;
+          uint8_t* dst = tiles + stage * C::STAGE_BYTES;
+#pragma unroll
+          for (int r = 0; r < C::CHUNKS; ++r) {
+            const int t = tok0 + 32 * r;
+            long long row = a.cache_rows;  // out of range: TMA fills zeros
+            if (t < L) {
+              if (a.block_table == nullptr) {
+                row = static_cast<long long>(s) * a.seq_stride + t;
+              } else {
+                const int pidx = t / a.page_size;
+                if (pidx < a.max_pages) {
+                  const int page = a.block_table[static_cast<long long>(s) * a.max_pages + pidx];
+                  row = static_cast<long long>(page) * a.page_size + t % a.page_size;
+                }
+              }
+              if (row < 0 || row >= a.cache_rows) row = a.cache_rows;
+            }
+            const int y = static_cast<int>(row);
+#pragma unroll
+            for (int d = 0; d < C::QK_BOXES; ++d) {
+              void* box = dst + d * C::BOX_BYTES + r * 4096;
+              if (d < C::QK_BOXES - 1)
+                tma_load_2d(box, &map_ckv, &full[stage], branch * C::W + 64 * d, y, policy);
+              else
+                tma_load_2d(box, &map_krope, &full[stage], 0, y, policy);
+            }
+          }
+        }
+      }
+      // Tail: every stage handed out must come back before the CTA may exit, so that no
+      // copy or MMA still targets this CTA's shared memory.
+      for (int k = max(0, it - STAGES); k < it; ++k) {
+        if (ok) {
+          if (!mbar_wait(&empty[k % STAGES], (k / STAGES) & 1, limit, abort_flag, status, 2)) ok = false;
+        }
+        if (!ok) {  // aborted: wait (bounded, ignoring the abort flag) for the copy itself
+          volatile int never = 0;
+          mbar_wait(&full[k % STAGES], (k / STAGES) & 1, limit, &never, status, 3);
+        }
+      }
+    }
+  } else if (warp == 9) {
+    // ------------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc_qk = idesc_f16_f32(128, NT, false);
+      const uint32_t tiles_addr = smem_u32(tiles);
+      int it = 0, seg = 0;
+      bool ok = true;
+      for (int s = s_first; ok && s < B && prefix[s] < t_end; ++s) {
+        const int j0 = max(t_begin, prefix[s]), j1 = min(t_end, prefix[s + 1]);
+        if (j0 >= j1) continue;
+        if (!mbar_wait(q_ready, seg & 1, limit, abort_flag, status, 10)) { ok = false; break; }
+        ++seg;
+        tc_fence_after();
+        for (int j = j0; j < j1; ++j, ++it) {
+          const int stage = it % STAGES;
+          if (!mbar_wait(&conv[stage], (it / STAGES) & 1, limit, abort_flag, status, 11)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t sb = it & 1;
+          const uint32_t k_base = tiles_addr + stage * C::STAGE_BYTES;
+#pragma unroll
+          for (int k = 0; k < C::QK_DIMS / 16; ++k) {
+            const uint64_t bdesc = smem_desc_sw128(k_base + (k >> 2) * C::BOX_BYTES + (k & 3) * 32, 16, 1024);
+            umma_f16_ts(tmem + C::TMEM_S + sb * NT, tmem + C::TMEM_Q + k * 8, bdesc, idesc_qk, k > 0 ? 1u : 0u);
+          }
+          umma_commit(&s_full[sb]);
+          if (j > j0) {
+            if (!mbar_wait(&p_ready[(it - 1) & 1], ((it - 1) >> 1) & 1, limit, abort_flag, status, 12)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            issue_pv<C>(tiles_addr, tmem, pv_done, empty, it - 1, j - 1 == j0, pv_box);
+          }
+        }
+        if (!ok) break;
+        if (!mbar_wait(&p_ready[(it - 1) & 1], ((it - 1) >> 1) & 1, limit, abort_flag, status, 13)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        issue_pv<C>(tiles_addr, tmem, pv_done, empty, it - 1, j1 - 1 == j0, pv_box);
+      }
+      if (!ok) {  // drain: let every MMA issued so far finish before TMEM is released
+        umma_commit(drain);
+        volatile int never = 0;
+        mbar_wait(drain, 0, limit, &never, status, 14);
+      }
+    }
+  } else if (warp >= 4) {
+    // ------------------------------------------------------------------ bf16 -> fp16
+    const int ct = threadIdx.x - 128;
+    int it = 0;
+    bool ok = true;
+    for (int s = s_first; ok && s < B && prefix[s] < t_end; ++s) {
+      const int j0 = max(t_begin, prefix[s]), j1 = min(t_end, prefix[s + 1]);
+      if (j0 >= j1) continue;
+      const int L = a.seq_lens[s];
+      for (int j = j0; j < j1; ++j, ++it) {
+        const int stage = it % STAGES;
+        if (!warp_wait(&full[stage], (it / STAGES) & 1, limit, abort_flag, status, 20)) { ok = false; break; }
+        const int n_valid = min(NT, L - (j - prefix[s]) * NT);
+        uint4* buf = reinterpret_cast<uint4*>(tiles + stage * C::STAGE_BYTES);
+        constexpr int N16 = C::STAGE_BYTES / 16;
+        static_assert(N16 % 128 == 0, "conversion split");
+#pragma unroll 1
+        for (int c0 = ct; c0 < N16; c0 += 128 * 4) {
+          uint4 v[4];
+#pragma unroll
+          for (int u = 0; u < 4; ++u)
+            if (c0 + u * 128 < N16) v[u] = buf[c0 + u * 128];
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            if (c0 + u * 128 >= N16) break;
+            const int row = ((c0 + u * 128) >> 3) % NT;
+            if (row < n_valid) {
+              v[u].x = bf16x2_to_f16x2(v[u].x);
+              v[u].y = bf16x2_to_f16x2(v[u].y);
+              v[u].z = bf16x2_to_f16x2(v[u].z);
+              v[u].w = bf16x2_to_f16x2(v[u].w);
+            } else {
+              v[u] = make_uint4(0u, 0u, 0u, 0u);
+            }
+            buf[c0 + u * 128] = v[u];
+          }
+        }
+        fence_proxy_async_smem();
+        mbar_arrive(&conv[stage]);
+      }
+    }
+  } else {
+    // ------------------------------------------------------------------ softmax + epilogue
+    const int row = threadIdx.x;                       // head row == TMEM lane
+    const uint32_t lane_addr = static_cast<uint32_t>(warp * 32) << 16;
+    const uint32_t t_row = tmem + lane_addr;
+    const float sl2 = a.scale_log2;
+    constexpr int kPChunk = NT >= 64 ? 64 : 32;  // tokens of P per TMEM store
+    int it = 0;
+    bool ok = true;
+    for (int s = s_first; ok && s < B && prefix[s] < t_end; ++s) {
+      const int j0 = max(t_begin, prefix[s]), j1 = min(t_end, prefix[s + 1]);
+      if (j0 >= j1) continue;
+      const int L = a.seq_lens[s];
+      // Q~ row of this head for branch `branch`: W latent columns then the 64 rope columns.
+      {
+        const uint4* qsrc = reinterpret_cast<const uint4*>(
+            a.q_tilde + (static_cast<long long>(s) * a.heads + min(row, a.heads - 1)) * 576);
+        const bool live = row < a.heads;
+        uint32_t w[32];
+#pragma unroll 1
+        for (int c = 0; c < C::QK_DIMS / 64; ++c) {
+          const int col0 = (c < C::QK_DIMS / 64 - 1) ? branch * C::W + 64 * c : 512;  // fp16 column
+#pragma unroll
+          for (int u = 0; u < 8; ++u) {
+            const uint4 v = live ? __ldg(qsrc + (col0 >> 3) + u) : make_uint4(0u, 0u, 0u, 0u);
+            w[4 * u + 0] = v.x; w[4 * u + 1] = v.y; w[4 * u + 2] = v.z; w[4 * u + 3] = v.w;
+          }
+          tmem_st32(t_row + C::TMEM_Q + 32 * c, w);
+        }
+        tmem_st_wait();
+        tc_fence_before();
+        mbar_arrive(q_ready);
+      }
+      float m_ref = -INFINITY, l = 0.f;
+      for (int j = j0; j < j1; ++j, ++it) {
+        const uint32_t sb = it & 1;
+        if (!warp_wait(&s_full[sb], (it >> 1) & 1, limit, abort_flag, status, 30)) { ok = false; break; }
+        tc_fence_after();
+        const int n_valid = min(NT, L - (j - prefix[s]) * NT);
+        uint32_t sr[NT];
+#pragma unroll
+        for (int k = 0; k < NT / 32; ++k) tmem_ld32(t_row + C::TMEM_S + sb * NT + 32 * k, sr + 32 * k);
+        tmem_ld_wait();
+        // scores in log2 units, masked past the sequence end (kept in the same registers)
+        float mt = -INFINITY;
+#pragma unroll
+        for (int k = 0; k < NT; ++k) {
+          const float xk = (k < n_valid) ? __uint_as_float(sr[k]) * sl2 : -INFINITY;
+          sr[k] = __float_as_uint(xk);
+          mt = fmaxf(mt, xk);
+        }
+        const bool first = (j == j0);
+        float factor = 1.f;
+        bool rescale = false;
+        if (first) {
+          m_ref = mt;
+        } else if (mt > m_ref + 8.f) {  // lazy rescale: keep the old reference unless it grew by 2^8
+          factor = ex2_approx(m_ref - mt);
+          m_ref = mt;
+          rescale = true;
+        }
+        float sum = 0.f;
+#pragma unroll
+        for (int k0 = 0; k0 < NT; k0 += kPChunk) {
+          // packed fp16 pairs overwrite score registers that are already consumed
+#pragma unroll
+          for (int k = 0; k < kPChunk / 2; ++k) {
+            const float p0 = ex2_approx(__uint_as_float(sr[k0 + 2 * k]) - m_ref);
+            const float p1 = ex2_approx(__uint_as_float(sr[k0 + 2 * k + 1]) - m_ref);
+            sum += p0 + p1;
+            sr[k0 / 2 + k] = pack_f16x2(p0, p1);
+          }
+          if constexpr (kPChunk == 64) tmem_st32(t_row + C::TMEM_S + sb * NT + k0 / 2, sr + k0 / 2);
+          else tmem_st16(t_row + C::TMEM_S + sb * NT + k0 / 2, sr + k0 / 2);
+        }
+        l = first ? sum : l * factor + sum;
+        if (!first) {
+          // O may only be touched once the previous tile's P*V has landed.
+          if (!warp_wait(pv_done, (it - 1) & 1, limit, abort_flag, status, 31)) { ok = false; break; }
+          tc_fence_after();
+          if (__any_sync(0xffffffffu, rescale)) {
+#pragma unroll 1
+            for (int k = 0; k < 4; ++k) {
+              uint32_t o[32];
+              tmem_ld32(t_row + C::TMEM_O + 32 * k, o);
+              tmem_ld_wait();
+#pragma unroll
+              for (int u = 0; u < 32; ++u) o[u] = __float_as_uint(__uint_as_float(o[u]) * factor);
+              tmem_st32(t_row + C::TMEM_O + 32 * k, o);
+            }
+          }
+        }
+        tmem_st_wait();
+        tc_fence_before();
+        mbar_arrive(&p_ready[sb]);
+      }
+      if (!ok) break;
+      // epilogue: the segment's last P*V must land before O is read
+      if (!warp_wait(pv_done, (it - 1) & 1, limit, abort_flag, status, 32)) { ok = false; break; }
+      tc_fence_after();
+      const long long slot = static_cast<long long>(g) + s;
+      float4* dst = reinterpret_cast<float4*>(a.o_part + ((slot * 4 + slice) * 128 + row) * 128);
+#pragma unroll 1
+      for (int k = 0; k < 4; ++k) {
+        uint32_t o[32];
+        tmem_ld32(t_row + C::TMEM_O + 32 * k, o);
+        tmem_ld_wait();
+        if (row < a.heads) {
+#pragma unroll
+          for (int u = 0; u < 8; ++u)
+            dst[k * 8 + u] = make_float4(__uint_as_float(o[4 * u]), __uint_as_float(o[4 * u + 1]),
+                                         __uint_as_float(o[4 * u + 2]), __uint_as_float(o[4 * u + 3]));
+        }
+      }
+      if (row < a.heads) a.ml_part[(slot * 4 + slice) * 128 + row] = make_float2(m_ref, l);
+      tc_fence_before();
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 9) {
+    tc_fence_after();
+    tmem_dealloc(tmem, C::TMEM_COLS);
+  }
+}
+
+template <int NB, int NT, int STAGES>
+cudaError_t launch_decode(const CUtensorMap& map_ckv, const CUtensorMap& map_krope, const DecodeArgs& a,
+                          int groups, cudaStream_t stream) {
+  using C = DecodeCfg<NB, NT, STAGES>;
+  auto kern = decode_kernel<NB, NT, STAGES>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
+  if (e != cudaSuccess) return e;
+  kern<<<dim3(4, groups), C::THREADS, C::SMEM_BYTES, stream>>>(map_ckv, map_krope, a);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+int decode_tile_tokens(int n_branch) { return n_branch == 4 ? 128 : (n_branch == 2 ? 64 : 32); }
+
+cudaError_t launch_decode_kernel(int n_branch, const CUtensorMap& map_ckv, const CUtensorMap& map_krope,
+                                 const DecodeArgs& a, int groups, cudaStream_t stream) {
+  switch (n_branch) {
+    case 4: return launch_decode<4, 128, 4>(map_ckv, map_krope, a, groups, stream);
+    case 2: return launch_decode<2, 64, 5>(map_ckv, map_krope, a, groups, stream);
+    case 1: return launch_decode<1, 32, 5>(map_ckv, map_krope, a, groups, stream);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+}  // namespace hra

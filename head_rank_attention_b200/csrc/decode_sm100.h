@@ -1,0 +1,36 @@
+// decode_sm100.h -- host-side interface of the split-KV decode kernel.
+#pragma once
+
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+
+namespace hra {
+
+// Arguments of one decode launch (device pointers; see hra.h for layouts).
+struct DecodeArgs {
+  const __half* q_tilde;      // fp16 [B, h, 576]: absorbed latent query (512) | rotated rope (64)
+  const int32_t* seq_lens;    // int32 [B]
+  const int32_t* block_table; // int32 [B, max_pages] or nullptr (contiguous layout)
+  int max_pages;
+  int page_size;
+  long long seq_stride;       // rows between sequences (contiguous layout)
+  long long cache_rows;       // rows addressable through the tensor maps
+  int batch;
+  int heads;
+  float scale_log2;           // softmax scale * log2(e)
+  float* o_part;              // fp32 [slots, 4, 128, 128]: un-normalised O per segment and slice
+  float2* ml_part;            // fp32 [slots, 4, 128] pairs: (running max in log2 units, row sum)
+  int* status;                // device status word
+  uint64_t wait_limit_ns;     // global-time budget of one device-side wait
+};
+
+// Tokens per cache tile for a branch count (decides the TMEM and shared-memory budget).
+int decode_tile_tokens(int n_branch);
+
+// Launch the decode kernel on grid (4 slices, `groups` KV splits).
+cudaError_t launch_decode_kernel(int n_branch, const CUtensorMap& map_ckv, const CUtensorMap& map_krope,
+                                 const DecodeArgs& a, int groups, cudaStream_t stream);
+
+}  // namespace hra

@@ -1,0 +1,138 @@
+/*
+ * hra.h -- C ABI of the B200 (sm_100a) latent-cache decode library (libhra.so).
+ *
+ * One call computes single-token decode attention for a batch of sequences over a
+ * compressed latent KV cache, in the three steps of "Multi-Head Low-Rank Attention"
+ * (section 方法步骤详情):
+ *   1. query-side absorption: q~^(b),(i) = alpha_q * alpha_kv * W_UK^(b),(i) q_nope^(i),
+ *      and RoPE on q_rope at position L-1;
+ *   2. MQA-style decode over the shared key [C_KV | K_RoPE] with value C_KV, with one
+ *      independent softmax per (head, branch); every branch reuses the shared K_RoPE;
+ *   3. output up-projection and branch sum:
+ *      out^(i) = branch_scale * alpha_kv * sum_b o_lat^(b),(i) W_UV^(b),(i).
+ * n_branch = 1 is MLA ("ML Revisit: Attention", Multi-Head Latent Attention: the
+ * absorbed QK^T = C_q W_q W_k^T C_kv^T with a decoupled RoPE key shared by all heads);
+ * n_branch = 4 is MLRA-4 (核心方法: O = sum_b Softmax(Q K_b^T) V_b).
+ * The softmax scale of every branch is 1/sqrt(d_nope + d_rope) by default
+ * ("vllbc02MLA", DeepseekV2Attention.__init__: scaling = qk_head_dim ** -0.5).
+ *
+ * Ownership: the caller owns every buffer.  The library allocates no device memory,
+ * keeps no pointer after a call returns, and runs asynchronously on `stream`.
+ * Errors: argument problems return a negative status before any launch, with a
+ * message from hra_last_error() (thread-local).  Launch failures return HRA_ERR_CUDA.
+ * Bounded device waits that expire write a status word in the workspace, read back
+ * by hra_check_device_status().
+ * Numerics: bf16 inputs; the tensor-core contractions run on fp16 operands (the cache
+ * tile is converted in shared memory, so |cache values| must stay below 65504) with
+ * fp32 accumulation; softmax, combine and up-projection in fp32.
+ */
+#ifndef HRA_H
+#define HRA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define HRA_API __attribute__((visibility("default")))
+#else
+#define HRA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  HRA_OK = 0,
+  HRA_ERR_INVALID_ARG = -1,     /* null/misaligned pointer, bad size or stride           */
+  HRA_ERR_UNSUPPORTED = -2,     /* shape outside the supported set (see below)           */
+  HRA_ERR_WORKSPACE = -3,       /* workspace missing or smaller than hra_workspace_size  */
+  HRA_ERR_CUDA = -4,            /* a CUDA runtime/driver call or a launch failed         */
+  HRA_ERR_DEVICE_TIMEOUT = -5   /* a bounded device-side wait expired                    */
+} hra_status;
+
+typedef enum { HRA_BF16 = 0, HRA_F32 = 1 } hra_dtype;
+
+/*
+ * Parameters of one decode step.  All pointers are device pointers, 16-byte aligned.
+ * Supported set: d_c = 512, d_rope = 64, d_nope = 128, d_v = 128, n_branch in {1,2,4},
+ * 1 <= num_heads <= 128, 1 <= batch <= 1024.
+ */
+typedef struct {
+  int batch;            /* B, number of sequences (one query token each)               */
+  int num_heads;        /* h, query heads sharing the latent cache                     */
+  int n_branch;         /* 1 = MLA, 2 = two-branch MLRA, 4 = MLRA-4                     */
+  int d_c, d_rope, d_nope, d_v;   /* 512, 64, 128, 128                                  */
+
+  const void* q;        /* bf16 [B, h, d_nope + d_rope], dense: q_nope | q_rope; q_rope is
+                           NOT rotated (the library rotates it at position seq_lens[b]-1) */
+  const void* ckv;      /* bf16 latent rows: row r is C_KV at ckv + r * ckv_stride          */
+  const void* krope;    /* bf16 RoPE-key rows, already rotated at their own positions:
+                           row r at krope + r * krope_stride.  A fused [rows, 576] cache
+                           is ckv = base, krope = base + 512, both strides 576            */
+  int64_t ckv_stride;   /* elements between consecutive rows; multiple of 8              */
+  int64_t krope_stride; /* elements between consecutive rows; multiple of 8              */
+  int64_t cache_rows;   /* rows addressable from ckv / krope (bounds every row access)   */
+
+  const int32_t* seq_lens;   /* int32 [B]: cached tokens per sequence, including the
+                                current one; 1 <= L.  L = 0 yields a zero output row    */
+  const int32_t* block_table;/* NULL: contiguous, row(b,t) = b * seq_stride + t.
+                                else int32 [B, max_pages]: row(b,t) =
+                                block_table[b*max_pages + t/page_size]*page_size + t%page_size */
+  int32_t max_pages;    /* columns of block_table                                       */
+  int32_t page_size;    /* rows per page; a multiple of 32                               */
+  int64_t seq_stride;   /* rows between sequences in the contiguous layout              */
+
+  const void* w_uk;     /* bf16 [h, d_c, d_nope]: W_UK[i] maps the latent to K_nope      */
+  const void* w_uv;     /* bf16 [h, d_c, d_v]:    W_UV[i] maps the latent to V            */
+  float alpha_q;        /* variance-correction scale on q_nope                          */
+  float alpha_kv;       /* variance-correction scale on the up-projected K_nope and V     */
+  float branch_scale;   /* scale on the branch sum (1/sqrt(n_branch) in the workloads)   */
+  float softmax_scale;  /* <= 0 selects 1/sqrt(d_nope + d_rope)                          */
+  float rope_theta;     /* RoPE base; pairs (j, j + d_rope/2) turn by pos*theta^(-2j/d_rope) */
+
+  void* out;            /* [B, h, d_v] in out_dtype                                      */
+  hra_dtype out_dtype;
+
+  void* workspace;      /* scratch of at least hra_workspace_size(p) bytes, 256-B aligned */
+  size_t workspace_bytes;
+  int num_splits;       /* KV splits = groups of 4 CTAs streaming disjoint token ranges;
+                           0 = one group per 4 SMs of the current device                 */
+  int wait_limit;       /* microseconds one device-side wait may last; 0 = 1 s           */
+  void* const* stage_events; /* optional, NULL = none: 4 caller-owned cudaEvent_t recorded on
+                                `stream` before absorption, before the split-KV decode, before
+                                the combine/up-projection and after it (per-stage timing)    */
+} hra_decode_params;
+
+/* Bytes of workspace one call with these parameters needs (0 on invalid parameters).
+ * Depends on batch, num_splits and the current device's SM count. */
+HRA_API size_t hra_workspace_size(const hra_decode_params* p);
+
+/* MLRA decode ("Multi-Head Low-Rank Attention", 方法步骤详情), n_branch in {1,2,4}. */
+HRA_API hra_status mlra_decode(const hra_decode_params* p, void* stream /* cudaStream_t */);
+
+/* MLA decode: the same call restricted to n_branch == 1 ("ML Revisit: Attention",
+ * Multi-Head Latent Attention; "vllbc02MLA", decode uses the absorbed MQA-like form). */
+HRA_API hra_status mla_decode(const hra_decode_params* p, void* stream /* cudaStream_t */);
+
+/* Synchronize `stream` and read the device status word of p->workspace.
+ * HRA_OK, or HRA_ERR_DEVICE_TIMEOUT if a bounded wait expired during the last call. */
+HRA_API hra_status hra_check_device_status(const hra_decode_params* p, void* stream);
+
+/* Self-test of the bounded-wait machinery: one block waits on an mbarrier that nothing
+ * arrives on, for at most `limit_us` microseconds (1..1e7), records the expiry in the
+ * status word of `workspace` and returns.  No copy or MMA is in flight.  Host code then
+ * reads the status with hra_check_device_status. */
+HRA_API hra_status hra_selftest_wait_timeout(void* workspace, int limit_us, void* stream);
+
+/* Message describing the last error on this thread ("" if none). */
+HRA_API const char* hra_last_error(void);
+
+/* Library version string. */
+HRA_API const char* hra_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* HRA_H */

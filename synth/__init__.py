@@ -74,6 +74,7 @@ class Workload:
     outlier_frac: float = 0.0     # fraction of positions whose whole cache row is scaled x8
     rope_theta: float = 10000.0
     seed: int = 0
+    lengths: Optional[tuple] = None  # explicit per-sequence lengths (overrides seq_len*)
 
     @property
     def sigma_o(self) -> float:
@@ -121,6 +122,9 @@ WORKLOADS = {
 
 def seq_lens(wl: Workload) -> np.ndarray:
     """Per-sequence lengths (int32 [B]); the query sits at position L-1."""
+    if wl.lengths is not None:
+        assert len(wl.lengths) == wl.batch
+        return np.asarray(wl.lengths, dtype=np.int32)
     if wl.seq_len_min is None:
         return np.full(wl.batch, wl.seq_len, dtype=np.int32)
     g = _gen(wl.seed, _T_LENS)
@@ -162,7 +166,7 @@ def page_table(wl: Workload) -> Optional[np.ndarray]:
     if wl.page_size == 0:
         return None
     lens = seq_lens(wl)
-    max_pages = int(-(-int(lens.max()) // wl.page_size))
+    max_pages = max(1, int(-(-int(lens.max()) // wl.page_size)))
     n_pages = wl.batch * max_pages
     perm = torch.randperm(n_pages, generator=_gen(wl.seed, _T_PAGES)).numpy().astype(np.int32)
     return perm.reshape(wl.batch, max_pages)
@@ -202,7 +206,7 @@ def make_inputs(wl: Workload, with_cache: bool = True) -> Inputs:
     bt = page_table(wl)
     w_uk, w_uv = weights(wl)
     q = queries(wl)
-    t_max = int(lens.max())
+    t_max = max(1, int(lens.max()))
     if bt is None:
         rows, seq_stride = wl.batch * t_max, t_max
     else:
@@ -239,3 +243,31 @@ def logical_rows(inp: Inputs, wl: Workload, s: int) -> torch.Tensor:
 def kv_bytes(lens) -> int:
     """Algorithmic KV-cache bytes one decode step reads: 576 bf16 per cached token."""
     return int(np.asarray(lens, dtype=np.int64).sum()) * ROW * 2
+
+
+@dataclasses.dataclass
+class DeviceInputs:
+    """Inputs copied to one device (same bytes as the host copy)."""
+    q: torch.Tensor
+    cache: torch.Tensor
+    seq_lens: torch.Tensor
+    block_table: Optional[torch.Tensor]
+    seq_stride: int
+    w_uk: torch.Tensor
+    w_uv: torch.Tensor
+
+    @property
+    def ckv(self) -> torch.Tensor:
+        return self.cache[:, :D_C]
+
+    @property
+    def krope(self) -> torch.Tensor:
+        return self.cache[:, D_C:]
+
+
+def to_device(inp: Inputs, device="cuda") -> DeviceInputs:
+    """Copy every input tensor to `device` unchanged."""
+    bt = None if inp.block_table is None else inp.block_table.to(device)
+    return DeviceInputs(q=inp.q.to(device), cache=inp.cache.to(device), seq_lens=inp.seq_lens.to(device),
+                        block_table=bt, seq_stride=inp.seq_stride, w_uk=inp.w_uk.to(device),
+                        w_uv=inp.w_uv.to(device))

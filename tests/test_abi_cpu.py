@@ -1,0 +1,111 @@
+"""CPU checks of the C-ABI library: it loads, exports every symbol include/hra.h declares,
+the ctypes mirror of hra_decode_params has the C layout, and argument validation
+returns the documented status before any CUDA call.  No compute runs here."""
+import ctypes
+import pathlib
+import re
+import subprocess
+
+import pytest
+
+import head_rank_attention_b200 as hra
+from head_rank_attention_b200 import _binding as B
+
+ROOT = pathlib.Path(__file__).resolve().parents[1]
+HEADER = ROOT / "include" / "hra.h"
+
+
+def _declared_symbols():
+    text = HEADER.read_text()
+    return sorted(set(re.findall(r"HRA_API\s+[\w\s\*]+?\b(\w+)\s*\(", text)))
+
+
+def test_library_loads_and_exports_every_declared_symbol():
+    lib = hra.load_library()
+    declared = _declared_symbols()
+    assert set(declared) == set(B.EXPORTS), declared
+    nm = subprocess.run(["nm", "-D", "--defined-only", str(hra.LIB_PATH)], capture_output=True, text=True, check=True)
+    exported = {line.split()[-1] for line in nm.stdout.splitlines() if " T " in line}
+    for name in declared:
+        assert name in exported, name
+        assert hasattr(lib, name)
+    assert "sm_100a" in hra.version()
+
+
+def test_params_layout_matches_c(tmp_path):
+    fields = [f[0] for f in B.HraDecodeParams._fields_]
+    prog = tmp_path / "layout.c"
+    lines = ['#include <stdio.h>', '#include <stddef.h>', '#include "hra.h"', 'int main(void) {',
+             '  printf("size %zu\\n", sizeof(hra_decode_params));']
+    lines += [f'  printf("{f} %zu\\n", offsetof(hra_decode_params, {f}));' for f in fields]
+    lines += ['  return 0;', '}']
+    prog.write_text("\n".join(lines))
+    exe = tmp_path / "layout"
+    subprocess.run(["gcc", "-std=c99", f"-I{ROOT / 'include'}", str(prog), "-o", str(exe)], check=True)
+    out = dict(line.split() for line in subprocess.run([str(exe)], capture_output=True, text=True,
+                                                        check=True).stdout.splitlines())
+    assert int(out["size"]) == ctypes.sizeof(B.HraDecodeParams)
+    for f in fields:
+        assert int(out[f]) == getattr(B.HraDecodeParams, f).offset, f
+
+
+def _fake_params(**over):
+    """Well-formed parameters with fake (aligned, never dereferenced) device pointers."""
+    p = B.HraDecodeParams()
+    p.batch, p.num_heads, p.n_branch = 2, 128, 4
+    p.d_c, p.d_rope, p.d_nope, p.d_v = 512, 64, 128, 128
+    p.q, p.ckv, p.krope, p.seq_lens = 0x10000, 0x20000, 0x20400, 0x30000
+    p.w_uk, p.w_uv, p.out = 0x40000, 0x50000, 0x60000
+    p.ckv_stride, p.krope_stride, p.cache_rows, p.seq_stride = 576, 576, 4096, 2048
+    p.alpha_q = p.alpha_kv = 1.0
+    p.branch_scale, p.softmax_scale, p.rope_theta = 0.5, 0.0, 10000.0
+    p.out_dtype = B.HRA_F32
+    p.num_splits = 37  # explicit: sizing then needs no device query
+    for k, v in over.items():
+        setattr(p, k, v)
+    return p
+
+
+def test_workspace_size_formula():
+    p = _fake_params()
+    n = hra.workspace_size(p)
+    slots = 37 + 2
+    expect = 256
+    expect = -(-(expect + 2 * 128 * 576 * 2) // 256) * 256
+    expect = -(-(expect + slots * 4 * 128 * 128 * 4) // 256) * 256
+    expect = -(-(expect + slots * 4 * 128 * 8) // 256) * 256
+    assert n == expect
+
+
+@pytest.mark.parametrize("over,status", [
+    (dict(q=0), B.HRA_ERR_INVALID_ARG),
+    (dict(ckv=0x20008), B.HRA_ERR_INVALID_ARG),          # misaligned
+    (dict(n_branch=3), B.HRA_ERR_UNSUPPORTED),
+    (dict(d_c=256), B.HRA_ERR_UNSUPPORTED),
+    (dict(num_heads=129), B.HRA_ERR_UNSUPPORTED),
+    (dict(batch=0), B.HRA_ERR_UNSUPPORTED),
+    (dict(ckv_stride=580), B.HRA_ERR_INVALID_ARG),        # not a multiple of 8
+    (dict(cache_rows=0), B.HRA_ERR_INVALID_ARG),
+    (dict(block_table=0x70000, max_pages=4, page_size=48), B.HRA_ERR_UNSUPPORTED),
+    (dict(out_dtype=7), B.HRA_ERR_INVALID_ARG),
+    (dict(rope_theta=0.0), B.HRA_ERR_INVALID_ARG),
+    (dict(workspace=0), B.HRA_ERR_WORKSPACE),
+    (dict(workspace=0x80000, workspace_bytes=1024), B.HRA_ERR_WORKSPACE),
+    (dict(workspace=0x80010, workspace_bytes=1 << 30), B.HRA_ERR_WORKSPACE),  # not 256-aligned
+])
+def test_validation_rejects_before_launch(over, status):
+    p = _fake_params(**over)
+    rc = hra.load_library().mlra_decode(ctypes.byref(p), None)
+    assert rc == status, hra.last_error()
+    assert hra.last_error() != ""
+
+
+def test_mla_decode_requires_one_branch():
+    p = _fake_params(n_branch=4)
+    with pytest.raises(hra.HraError) as e:
+        hra.mla_decode(p, stream=0)
+    assert e.value.status == B.HRA_ERR_INVALID_ARG
+
+
+def test_workspace_size_zero_on_invalid():
+    assert hra.load_library().hra_workspace_size(ctypes.byref(_fake_params(n_branch=5))) == 0

@@ -1,0 +1,170 @@
+"""GPU parity: the CUDA path (through the C ABI) against the fp64 oracle on the same
+seeded inputs.  Small cases are compared element by element over every output; the five
+full-size workloads are compared on sampled (sequence, head) outputs in the launch
+configuration the benchmark uses (num_splits = 0: one split per 4 SMs)."""
+import numpy as np
+import pytest
+import torch
+
+import head_rank_attention_b200 as hra
+import oracle
+import synth
+from gpu_cases import assert_parity, run_gpu
+
+pytestmark = pytest.mark.gpu
+
+if torch.cuda.is_available():
+    torch.backends.cuda.matmul.allow_tf32 = False
+
+
+def _case(name, n_branch, lengths, heads=128, page_size=0, **kw):
+    return synth.Workload(name, n_branch, len(lengths), heads, max(lengths), page_size=page_size,
+                          lengths=tuple(lengths), **kw)
+
+
+TAILS = (1, 31, 32, 33, 127, 128, 129, 1000)
+
+SMALL = [
+    _case("tails_mlra4", 4, TAILS),
+    _case("tails_mlra2", 2, TAILS),
+    _case("tails_mla", 1, TAILS),
+    _case("paged64_mlra4", 4, (5, 64, 65, 700), page_size=64),
+    _case("paged32_mlra2", 2, (5, 64, 65, 700), page_size=32),
+    _case("paged128_mla", 1, (5, 64, 65, 700), page_size=128),
+    _case("h1_mlra4", 4, (77, 300), heads=1),
+    _case("h16_mlra4", 4, (2048,), heads=16, alpha_q=2048 ** 0.5 / 1536 ** 0.5, alpha_kv=2.0, branch_scale=0.5),
+    _case("h100_mla", 1, (513, 9), heads=100),
+    _case("stress_mlra4", 4, (3000, 17), alpha_q=synth.A_Q_V3, alpha_kv=synth.A_KV_V3),
+    _case("stress_mla", 1, (3000, 17), alpha_q=synth.A_Q_V3, alpha_kv=synth.A_KV_V3),
+    _case("outlier_mlra4", 4, (5000,), outlier_frac=0.01),
+]
+
+
+@pytest.mark.parametrize("wl", SMALL, ids=lambda w: w.name)
+def test_small_full_parity(wl):
+    inp = synth.make_inputs(wl)
+    dev = synth.to_device(inp)
+    out, _, _ = run_gpu(dev, wl)
+    ref = oracle.decode_batch(inp, wl, form="absorbed")
+    assert_parity(out.cpu().numpy(), ref, wl.name)
+
+
+@pytest.mark.parametrize("num_splits", [1, 3, 37, 200])
+def test_split_count_invariance(num_splits):
+    """Any partition of the token stream across splits gives the same result (LSE combine)."""
+    wl = _case("splits", 4, (1, 130, 2000, 64))
+    inp = synth.make_inputs(wl)
+    dev = synth.to_device(inp)
+    ref = oracle.decode_batch(inp, wl, form="absorbed")
+    out, _, _ = run_gpu(dev, wl, num_splits=num_splits)
+    assert_parity(out.cpu().numpy(), ref, f"splits={num_splits}")
+
+
+def test_many_sequences():
+    """B=300 short sequences: many sequences per split, prefix scan over > 32 lengths."""
+    rng = np.random.default_rng(5)
+    wl = _case("many", 4, tuple(int(x) for x in rng.integers(1, 200, size=300)), heads=8)
+    inp = synth.make_inputs(wl)
+    out, _, _ = run_gpu(synth.to_device(inp), wl)
+    assert_parity(out.cpu().numpy(), oracle.decode_batch(inp, wl, form="absorbed"), "many")
+
+
+def test_bf16_output():
+    wl = _case("bf16out", 4, (700, 33))
+    inp = synth.make_inputs(wl)
+    out, _, _ = run_gpu(synth.to_device(inp), wl, out_dtype=torch.bfloat16)
+    assert_parity(out.float().cpu().numpy(), oracle.decode_batch(inp, wl, form="absorbed"), "bf16 out")
+
+
+def test_paged_equals_contiguous_bitwise():
+    """Same logical cache, paged (random page table) or contiguous: identical bits."""
+    lens = (100, 640, 33)
+    wl_c = _case("layout", 4, lens)
+    wl_p = _case("layout", 4, lens, page_size=32)
+    out_c, _, _ = run_gpu(synth.to_device(synth.make_inputs(wl_c)), wl_c)
+    out_p, _, _ = run_gpu(synth.to_device(synth.make_inputs(wl_p)), wl_p)
+    assert torch.equal(out_c, out_p)
+
+
+def test_mla_entry_point_and_determinism():
+    wl = _case("mla_api", 1, (900, 5))
+    dev = synth.to_device(synth.make_inputs(wl))
+    a, _, _ = run_gpu(dev, wl, api="mla")
+    b, _, _ = run_gpu(dev, wl, api="mlra")
+    c, _, _ = run_gpu(dev, wl, api="mlra")
+    assert torch.equal(a, b) and torch.equal(b, c)
+
+
+def test_mlra4_differs_from_mla_on_gpu():
+    """Guards against a kernel that sums branch keys before the softmax."""
+    lens = (1500,)
+    wl4 = _case("neg", 4, lens, branch_scale=1.0)
+    wl1 = _case("neg", 1, lens)
+    inp = synth.make_inputs(wl4)
+    dev = synth.to_device(inp)
+    o4, _, _ = run_gpu(dev, wl4)
+    o1, _, _ = run_gpu(dev, wl1)
+    assert (o4 - o1).abs().max() > 0.1 * o1.abs().max()
+
+
+def test_zero_length_sequence_gives_zero_row():
+    wl = _case("zero", 4, (0, 50))
+    inp = synth.make_inputs(wl)
+    out, _, _ = run_gpu(synth.to_device(inp), wl)
+    assert torch.all(out[0] == 0)
+    ref = oracle.decode_batch(inp, wl, seqs=[1], form="absorbed")
+    assert_parity(out[1:].cpu().numpy(), ref, "zero-length neighbour")
+
+
+def test_bounded_wait_reports_timeout_and_context_survives():
+    """A wait that nothing satisfies ends with HRA_ERR_DEVICE_TIMEOUT; the next call works."""
+    wl = _case("timeout", 4, (200,))
+    inp = synth.make_inputs(wl)
+    dev = synth.to_device(inp)
+    out, p, ws = run_gpu(dev, wl)
+    hra.selftest_wait_timeout(ws, limit_us=2000)
+    with pytest.raises(hra.HraError) as e:
+        hra.check_device_status(p)
+    assert e.value.status == hra._binding.HRA_ERR_DEVICE_TIMEOUT
+    out2, _, _ = run_gpu(dev, wl, workspace=ws)
+    assert torch.equal(out, out2)
+
+
+# ---- the five workloads at full size -------------------------------------------------------
+
+_FULL_CACHE = {}
+
+
+def _full_inputs(wl):
+    key = (wl.batch, wl.heads, wl.seq_len, wl.seq_len_min, wl.page_size, wl.outlier_frac, wl.n_branch)
+    if key not in _FULL_CACHE:
+        _FULL_CACHE.clear()
+        torch.cuda.empty_cache()
+        inp = synth.make_inputs(wl)
+        _FULL_CACHE[key] = (inp, synth.to_device(inp))
+    return _FULL_CACHE[key]
+
+
+FULL = [
+    ("small_mlra4_h16_t2k", None, None),           # every output, expanded definition
+    ("mla_b32_t8k", [0, 13, 31], None),
+    ("paged_b64_t32k_mlra4", [0, 37, 63], list(range(0, 128, 8))),
+    ("paged_b64_t32k_mlra2", [0, 37, 63], list(range(0, 128, 8))),
+    ("paged_b64_t32k_mla", [0, 37, 63], list(range(0, 128, 8))),
+    ("long_mlra4_b4_t64k_128k", None, list(range(0, 128, 8))),
+    ("vlong_mlra4_b1_t2m", None, list(range(0, 128, 16))),
+]
+
+
+@pytest.mark.parametrize("name,seqs,heads", FULL, ids=[f[0] for f in FULL])
+def test_full_size_workload(name, seqs, heads):
+    wl = synth.WORKLOADS[name]
+    inp, dev = _full_inputs(wl)
+    out, _, _ = run_gpu(dev, wl)
+    got = out.cpu().numpy()
+    assert np.isfinite(got).all()
+    seqs = list(range(wl.batch)) if seqs is None else seqs
+    heads_idx = list(range(wl.heads)) if heads is None else heads
+    form = "expanded" if name == "small_mlra4_h16_t2k" else "absorbed"
+    ref = oracle.decode_batch(inp, wl, heads=heads_idx, seqs=seqs, form=form)
+    assert_parity(got[np.ix_(seqs, heads_idx)], ref, name)
