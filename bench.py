@@ -228,7 +228,12 @@ def run_native(args, wl, world, rank, local):
 
     # per-step stage events: [before absorb, before decode, before combine, after combine]
     events = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    for evs in events:  # torch creates the underlying cudaEvent_t on first record
+        for e in evs:
+            e.record(stream)
+    torch.cuda.synchronize()
     handles = [(ctypes.c_void_p * 4)(*[e.cuda_event for e in evs]) for evs in events]
+    assert all(h for hs in handles for h in hs), "CUDA events were not created
 
     for _ in range(args.warmup):
         hra.mlra_decode(p, stream)

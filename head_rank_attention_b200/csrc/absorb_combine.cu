@@ -114,11 +114,16 @@ __global__ void __launch_bounds__(256) combine_upproj_kernel(const CombineArgs a
     if (prefix[seq + 1] > prefix[seq]) {
       const int g_lo = group_of_tile(prefix[seq], G, T);
       const int g_hi = group_of_tile(prefix[seq + 1] - 1, G, T);
+      // Every group between g_lo and g_hi that owns at least one tile streamed part of this
+      // sequence; groups with an empty range (more groups than tiles) wrote nothing.
       float M = -INFINITY;
-      for (int g = g_lo; g <= g_hi; ++g)
+      for (int g = g_lo; g <= g_hi; ++g) {
+        if (group_tile_begin(g, G, T) == group_tile_begin(g + 1, G, T)) continue;
         M = fmaxf(M, a.ml_part[((static_cast<long long>(g) + seq) * 4 + slice) * 128 + i].x);
+      }
       float den = 0.f;
       for (int g = g_lo; g <= g_hi; ++g) {
+        if (group_tile_begin(g, G, T) == group_tile_begin(g + 1, G, T)) continue;
         const long long slot = static_cast<long long>(g) + seq;
         const float2 ml = a.ml_part[(slot * 4 + slice) * 128 + i];
         const float wgt = exp2f(ml.x - M);

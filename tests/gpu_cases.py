@@ -14,7 +14,7 @@ MEAN_REL = 2e-3     # sum|g - r| / sum|r| <= MEAN_REL
 
 
 def run_gpu(dev: synth.DeviceInputs, wl: synth.Workload, *, out_dtype=torch.float32, num_splits: int = 0,
-            api: str = "mlra", workspace=None):
+            api: str = "mlra", workspace=None, poison: bool = True):
     B, h = dev.q.shape[0], dev.q.shape[1]
     out = torch.empty(B, h, synth.D_V, dtype=out_dtype, device=dev.q.device)
     p = hra.make_params(dev.q, dev.ckv, dev.krope, dev.seq_lens, dev.w_uk, dev.w_uv, out,
@@ -25,6 +25,8 @@ def run_gpu(dev: synth.DeviceInputs, wl: synth.Workload, *, out_dtype=torch.floa
     ws = hra.alloc_workspace(p) if workspace is None else workspace
     if workspace is not None:
         p.workspace, p.workspace_bytes = ws.data_ptr(), ws.numel()
+    if poison:  # NaN bytes everywhere: any read of a slot the call did not write shows up
+        ws.fill_(0xFF)
     (hra.mla_decode if api == "mla" else hra.mlra_decode)(p)
     hra.check_device_status(p)
     return out, p, ws
