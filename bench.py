@@ -79,62 +79,59 @@ def ncu_traffic(workload: str):
 
 
 class ClockSampler:
-    """nvidia-smi clock/throttle sampling during the timed region."""
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    """SM clock and throttle-reason sampling during the timed region, in-process through
+    NVML every 2 ms (a background thread), so short timed regions still get samples."""
+    REASONS = {"hw_slowdown": 0x8, "sw_thermal_slowdown": 0x20, "hw_thermal_slowdown": 0x40,
+               "sw_power_cap": 0x4}
 
     def __init__(self, device: int):
-        self.gpu = str(device)
-        try:  # address the GPU by UUID so CUDA_VISIBLE_DEVICES remapping cannot mislead nvidia-smi
-            u = str(torch.cuda.get_device_properties(device).uuid)
-            self.gpu = u if u.startswith("GPU-") else "GPU-" + u
-        except Exception:
-            pass
-        self.proc = None
+        self.device = device
+        self.samples = []
+        self.max_mhz = None
+        self._stop = None
 
     def __enter__(self):
+        import threading
         try:
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
-        except (OSError, FileNotFoundError):
-            self.proc = None
-        time.sleep(0.3)
+            import pynvml
+            pynvml.nvmlInit()
+            uuid = str(torch.cuda.get_device_properties(self.device).uuid)
+            uuid = uuid if uuid.startswith("GPU-") else "GPU-" + uuid
+            try:
+                h = pynvml.nvmlDeviceGetHandleByUUID(uuid)
+            except Exception:
+                h = pynvml.nvmlDeviceGetHandleByIndex(self.device)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM)
+        except Exception:
+            return self
+        self._stop = threading.Event()
+
+        def run():
+            while not self._stop.is_set():
+                try:
+                    clk = pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM)
+                    rs = pynvml.nvmlDeviceGetCurrentClocksEventReasons(h)
+                    self.samples.append((clk, rs))
+                except Exception:
+                    pass
+                self._stop.wait(0.002)
+
+        self._thread = threading.Thread(target=run, daemon=True)
+        self._thread.start()
         return self
 
     def __exit__(self, *exc):
-        self.lines = []
-        if self.proc is not None:
-            time.sleep(0.2)
-            self.proc.terminate()
-            try:
-                out, _ = self.proc.communicate(timeout=5)
-            except subprocess.TimeoutExpired:
-                self.proc.kill()
-                out, _ = self.proc.communicate()
-            self.lines = [l for l in out.splitlines() if l.strip()]
+        if self._stop is not None:
+            self._stop.set()
+            self._thread.join(timeout=2)
 
     def summary(self):
-        sm, mx, reasons = [], [], set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for l in self.lines:
-            f = [x.strip() for x in l.split(",")]
-            if len(f) < 9:
-                continue
-            try:
-                sm.append(float(f[1]))
-                mx.append(float(f[2]))
-            except ValueError:
-                continue
-            for n, v in zip(names, f[5:9]):
-                if v.lower().startswith("active"):
-                    reasons.add(n)
-        if not sm:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
-        loaded = sorted(sm)[len(sm) // 4:] or sm  # drop the idle tail at the edges
-        return {"sm_mhz": statistics.median(loaded), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
-                "samples": len(sm)}
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": ["unsampled"]}
+        clks = sorted(c for c, _ in self.samples)
+        reasons = sorted({n for _, r in self.samples for n, bit in self.REASONS.items() if r & bit})
+        return {"sm_mhz": statistics.median(clks), "sm_max_mhz": self.max_mhz, "sm_mhz_min": clks[0],
+                "reasons": reasons, "samples": len(clks), "source": "NVML, 2 ms period, timed region only"}
 
 
 def time_oracle_sample(wl: synth.Workload, n_seqs: int, n_heads: int):
@@ -233,7 +230,7 @@ def run_native(args, wl, world, rank, local):
             e.record(stream)
     torch.cuda.synchronize()
     handles = [(ctypes.c_void_p * 4)(*[e.cuda_event for e in evs]) for evs in events]
-    assert all(h for hs in handles for h in hs), "CUDA events were not created
+    assert all(h for hs in handles for h in hs), "CUDA events were not created"
 
     for _ in range(args.warmup):
         hra.mlra_decode(p, stream)

@@ -12,7 +12,8 @@ struct AbsorbArgs {
   const __nv_bfloat16* q;     // [B, h, 192]
   const __nv_bfloat16* w_uk;  // [h, 512, 128]
   const int32_t* seq_lens;    // [B]
-  __half* q_tilde;            // [B, h, 576] out
+  __half* q_tilde;            // out: fp16 [B, h, 576], or (two_term) bf16 hi [B, h, 576] + bf16 lo [B, h, 576]
+  int two_term;               // 1: store q~ as bf16 hi + bf16 lo (MLRA-4 kernel); 0: fp16
   int* status;                // cleared by this kernel (first kernel of a call)
   int batch, heads;
   float alpha_q, alpha_kv, rope_theta;

@@ -112,7 +112,7 @@ hra_status make_plan(const hra_decode_params* p, Plan* plan) {
   plan->slots = static_cast<long long>(plan->groups) + p->batch;
   size_t off = 256;  // device status word
   plan->q_tilde = off;
-  off = round256(off + static_cast<size_t>(p->batch) * p->num_heads * 576 * sizeof(__half));
+  off = round256(off + 2 * static_cast<size_t>(p->batch) * p->num_heads * 576 * sizeof(__half));  // up to two terms
   plan->o_part = off;
   off = round256(off + static_cast<size_t>(plan->slots) * 4 * 128 * 128 * sizeof(float));
   plan->ml_part = off;
@@ -179,6 +179,7 @@ hra_status run_decode(const hra_decode_params* p, cudaStream_t stream) {
   ab.alpha_q = p->alpha_q;
   ab.alpha_kv = p->alpha_kv;
   ab.rope_theta = p->rope_theta;
+  ab.two_term = p->n_branch == 4 ? 1 : 0;
   e = hra::launch_absorb_q(ab, stream);
   if (e != cudaSuccess) return cuda_fail(e, "absorb_q launch");
 

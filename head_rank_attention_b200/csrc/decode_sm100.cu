@@ -12,14 +12,18 @@
 // A CTA streams, for every tile of NT tokens, the branch's W latent columns plus the 64
 // RoPE columns (TMA, 64x32 boxes, 128-byte swizzle), converts them to fp16 in shared
 // memory, computes S = Q~_b [C_b | K_R]^T for all 128 head rows with tcgen05 (A = Q~
-// from TMEM, B = the tile, D = S in TMEM), runs the online softmax with one thread per
-// head row, writes P (fp16) back over S in TMEM and accumulates O += P V with V = its
-// 128 latent columns of the same tile (A = P from TMEM, B = MN-major tile).  Each
-// segment ends by writing the un-normalised O row, the running max m (log2 units) and
-// the row sum l of every head to the workspace.
+// from TMEM, B = the tile, D = S in TMEM), runs the online softmax, writes P (fp16) back
+// over S in TMEM and accumulates O += P V with V = its 128 latent columns of the same
+// tile (A = P from TMEM, B = MN-major tile).  Each segment ends by writing the
+// un-normalised O row, the running max m (log2 units) and the row sum l of every head.
 //
-// Warp roles: warps 0-3 softmax + epilogue (thread = head row = TMEM lane), warps 4-7
-// bf16 -> fp16 conversion, warp 8 TMA producer, warp 9 TMEM allocator + MMA issuer.
+// Warp roles (14 warps):
+//   0-3   softmax half 0: TMEM lane = head row, score columns [0, NT/2), O columns [0, 64)
+//   4-7   softmax half 1: same rows, score columns [NT/2, NT), O columns [64, 128)
+//         (the two halves agree on every row's running max through shared memory)
+//   8-11  bf16 -> fp16 conversion of each arrived tile (zeroing rows past the end)
+//   12    TMA producer
+//   13    TMEM allocator + MMA issuer (one elected thread)
 // Every wait is bounded (see sm100.cuh); on expiry the CTA drains and exits with the
 // failure recorded in the workspace status word.
 
@@ -42,12 +46,16 @@ struct DecodeCfg {
   static constexpr int BOX_BYTES = NT * 128;         // one 64-column box over NT rows
   static constexpr int STAGE_BYTES = QK_BOXES * BOX_BYTES;
   static constexpr int CHUNKS = NT / 32;             // TMA row chunks per tile
+  static constexpr int HALF = NT / 2;                // score columns per softmax thread
   static constexpr int TMEM_O = 0;                   // O: 128 fp32 columns
   static constexpr int TMEM_S = 128;                 // S/P double buffer: 2 x NT columns
   static constexpr int TMEM_Q = 128 + 2 * NT;        // Q~ (fp16 pairs): QK_DIMS/2 columns
   static constexpr int TMEM_COLS = 512;
-  static constexpr int THREADS = 320;
-  static constexpr int MISC_BYTES = 256 + 4 * (kMaxBatch + 1);
+  static constexpr int THREADS = 448;
+  // shared memory after the tile stages: barriers | row-max/row-sum exchange | tile prefix
+  static constexpr int BAR_BYTES = 512;
+  static constexpr int RED_BYTES = (2 * 2 * 128 + 2 * 128) * 4;
+  static constexpr int MISC_BYTES = BAR_BYTES + RED_BYTES + 4 * (kMaxBatch + 1);
   static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + MISC_BYTES;
   static_assert(TMEM_Q + QK_DIMS / 2 <= TMEM_COLS, "TMEM budget");
   static_assert(NT % 32 == 0 && NT >= 32 && NT <= 256, "tile rows");
@@ -56,12 +64,14 @@ struct DecodeCfg {
 
 namespace {
 
+constexpr uint32_t kFull = 0xffffffffu;
+
 // All lanes of a warp poll; the result is made warp-uniform so that the .sync.aligned
 // tcgen05 instructions and warp votes that follow see a converged warp.
 __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, uint64_t limit, volatile int* abort,
                                           int* status, int where) {
   const bool ok = mbar_wait(bar, parity, limit, abort, status, where);
-  return __all_sync(0xffffffffu, ok);
+  return __all_sync(kFull, ok);
 }
 
 // Smallest sequence index s with prefix[s + 1] > t.
@@ -95,23 +105,28 @@ __device__ __forceinline__ void issue_pv(uint32_t tiles_addr, uint32_t tmem, uin
 }
 
 template <int NB, int NT, int STAGES>
-__global__ void __launch_bounds__(320, 1)
+__global__ void __launch_bounds__(448, 1)
 decode_kernel(const __grid_constant__ CUtensorMap map_ckv, const __grid_constant__ CUtensorMap map_krope,
               const DecodeArgs a) {
   using C = DecodeCfg<NB, NT, STAGES>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* tiles = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint64_t* full = reinterpret_cast<uint64_t*>(tiles + STAGES * C::STAGE_BYTES);
+  uint8_t* misc = tiles + STAGES * C::STAGE_BYTES;
+  uint64_t* full = reinterpret_cast<uint64_t*>(misc);
   uint64_t* conv = full + STAGES;
   uint64_t* empty = conv + STAGES;
   uint64_t* s_full = empty + STAGES;  // [2]
   uint64_t* p_ready = s_full + 2;     // [2]
-  uint64_t* pv_done = p_ready + 2;
+  uint64_t* red_bar = p_ready + 2;    // [2] row-max exchange, alternating per tile
+  uint64_t* lsum_bar = red_bar + 2;   // row-sum exchange, once per segment
+  uint64_t* pv_done = lsum_bar + 1;
   uint64_t* q_ready = pv_done + 1;
   uint64_t* drain = q_ready + 1;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-  int* prefix = reinterpret_cast<int*>(tiles + STAGES * C::STAGE_BYTES + 256);
+  float* red_max = reinterpret_cast<float*>(misc + C::BAR_BYTES);  // [2 buf][2 half][128]
+  float* red_l = red_max + 2 * 2 * 128;                              // [2 half][128]
+  int* prefix = reinterpret_cast<int*>(misc + C::BAR_BYTES + C::RED_BYTES);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -133,19 +148,21 @@ decode_kernel(const __grid_constant__ CUtensorMap map_ckv, const __grid_constant
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&s_full[i], 1);
-      mbar_init(&p_ready[i], 128);
+      mbar_init(&p_ready[i], 256);
+      mbar_init(&red_bar[i], 256);
     }
+    mbar_init(lsum_bar, 256);
     mbar_init(pv_done, 1);
-    mbar_init(q_ready, 128);
+    mbar_init(q_ready, 256);
     mbar_init(drain, 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
-  if (warp == 9) {
+  if (warp == 13) {
     tmem_alloc(tmem_slot, C::TMEM_COLS);
     tmem_relinquish();
   }
-  if (warp == 8 && lane == 0) {
+  if (warp == 12 && lane == 0) {
     tma_prefetch_desc(&map_ckv);
     tma_prefetch_desc(&map_krope);
   }
@@ -159,7 +176,7 @@ decode_kernel(const __grid_constant__ CUtensorMap map_ckv, const __grid_constant
   const int t_end = T > 0 ? group_tile_begin(g + 1, G, T) : 0;
   const int s_first = (t_begin < t_end) ? first_seq(prefix, B, t_begin) : B;
 
-  if (warp == 8) {
+  if (warp == 12) {
     // ------------------------------------------------------------------ TMA producer
     if (lane == 0) {
       const uint64_t policy = l2_policy_evict_first();
@@ -219,7 +236,7 @@ decode_kernel(const __grid_constant__ CUtensorMap map_ckv, const __grid_constant
         }
       }
     }
-  } else if (warp == 9) {
+  } else if (warp == 13) {
     // ------------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       constexpr uint32_t idesc_qk = idesc_f16_f32(128, NT, false);
@@ -267,9 +284,11 @@ decode_kernel(const __grid_constant__ CUtensorMap map_ckv, const __grid_constant
         mbar_wait(drain, 0, limit, &never, status, 14);
       }
     }
-  } else if (warp >= 4) {
+  } else if (warp >= 8) {
     // ------------------------------------------------------------------ bf16 -> fp16
-    const int ct = threadIdx.x - 128;
+    const int ct = threadIdx.x - 256;
+    constexpr int N16 = C::STAGE_BYTES / 16;
+    static_assert(N16 % 128 == 0, "conversion split");
     int it = 0;
     bool ok = true;
     for (int s = s_first; ok && s < B && prefix[s] < t_end; ++s) {
@@ -281,27 +300,37 @@ decode_kernel(const __grid_constant__ CUtensorMap map_ckv, const __grid_constant
         if (!warp_wait(&full[stage], (it / STAGES) & 1, limit, abort_flag, status, 20)) { ok = false; break; }
         const int n_valid = min(NT, L - (j - prefix[s]) * NT);
         uint4* buf = reinterpret_cast<uint4*>(tiles + stage * C::STAGE_BYTES);
-        constexpr int N16 = C::STAGE_BYTES / 16;
-        static_assert(N16 % 128 == 0, "conversion split");
-#pragma unroll 1
-        for (int c0 = ct; c0 < N16; c0 += 128 * 4) {
-          uint4 v[4];
+        if (n_valid == NT) {
+#pragma unroll 2
+          for (int c0 = ct; c0 < N16; c0 += 128 * 4) {
+            uint4 v[4];
 #pragma unroll
-          for (int u = 0; u < 4; ++u)
-            if (c0 + u * 128 < N16) v[u] = buf[c0 + u * 128];
+            for (int u = 0; u < 4; ++u)
+              if (c0 + u * 128 < N16) v[u] = buf[c0 + u * 128];
 #pragma unroll
-          for (int u = 0; u < 4; ++u) {
-            if (c0 + u * 128 >= N16) break;
-            const int row = ((c0 + u * 128) >> 3) % NT;
-            if (row < n_valid) {
-              v[u].x = bf16x2_to_f16x2(v[u].x);
-              v[u].y = bf16x2_to_f16x2(v[u].y);
-              v[u].z = bf16x2_to_f16x2(v[u].z);
-              v[u].w = bf16x2_to_f16x2(v[u].w);
-            } else {
-              v[u] = make_uint4(0u, 0u, 0u, 0u);
+            for (int u = 0; u < 4; ++u) {
+              if (c0 + u * 128 < N16) {
+                v[u].x = bf16x2_to_f16x2(v[u].x);
+                v[u].y = bf16x2_to_f16x2(v[u].y);
+                v[u].z = bf16x2_to_f16x2(v[u].z);
+                v[u].w = bf16x2_to_f16x2(v[u].w);
+                buf[c0 + u * 128] = v[u];
+              }
             }
-            buf[c0 + u * 128] = v[u];
+          }
+        } else {
+#pragma unroll 1
+          for (int c = ct; c < N16; c += 128) {
+            const int row = (c >> 3) % NT;
+            uint4 v = make_uint4(0u, 0u, 0u, 0u);
+            if (row < n_valid) {
+              v = buf[c];
+              v.x = bf16x2_to_f16x2(v.x);
+              v.y = bf16x2_to_f16x2(v.y);
+              v.z = bf16x2_to_f16x2(v.z);
+              v.w = bf16x2_to_f16x2(v.w);
+            }
+            buf[c] = v;
           }
         }
         fence_proxy_async_smem();
@@ -310,25 +339,27 @@ decode_kernel(const __grid_constant__ CUtensorMap map_ckv, const __grid_constant
     }
   } else {
     // ------------------------------------------------------------------ softmax + epilogue
-    const int row = threadIdx.x;                       // head row == TMEM lane
-    const uint32_t lane_addr = static_cast<uint32_t>(warp * 32) << 16;
+    constexpr int HALF = C::HALF;
+    const int half = warp >> 2;                        // which half of the score columns
+    const int row = threadIdx.x & 127;                 // head row == TMEM lane
+    const uint32_t lane_addr = static_cast<uint32_t>((warp & 3) * 32) << 16;
     const uint32_t t_row = tmem + lane_addr;
     const float sl2 = a.scale_log2;
-    constexpr int kPChunk = NT >= 64 ? 64 : 32;  // tokens of P per TMEM store
-    int it = 0;
+    int it = 0, seg = 0;
     bool ok = true;
     for (int s = s_first; ok && s < B && prefix[s] < t_end; ++s) {
       const int j0 = max(t_begin, prefix[s]), j1 = min(t_end, prefix[s + 1]);
       if (j0 >= j1) continue;
       const int L = a.seq_lens[s];
-      // Q~ row of this head for branch `branch`: W latent columns then the 64 rope columns.
+      // Q~ row of this head for branch `branch`: W latent columns then the 64 rope columns;
+      // the two halves store alternate 64-column chunks.
       {
         const uint4* qsrc = reinterpret_cast<const uint4*>(
             a.q_tilde + (static_cast<long long>(s) * a.heads + min(row, a.heads - 1)) * 576);
         const bool live = row < a.heads;
         uint32_t w[32];
 #pragma unroll 1
-        for (int c = 0; c < C::QK_DIMS / 64; ++c) {
+        for (int c = half; c < C::QK_DIMS / 64; c += 2) {
           const int col0 = (c < C::QK_DIMS / 64 - 1) ? branch * C::W + 64 * c : 512;  // fp16 column
 #pragma unroll
           for (int u = 0; u < 8; ++u) {
@@ -347,18 +378,30 @@ decode_kernel(const __grid_constant__ CUtensorMap map_ckv, const __grid_constant
         if (!warp_wait(&s_full[sb], (it >> 1) & 1, limit, abort_flag, status, 30)) { ok = false; break; }
         tc_fence_after();
         const int n_valid = min(NT, L - (j - prefix[s]) * NT);
-        uint32_t sr[NT];
-#pragma unroll
-        for (int k = 0; k < NT / 32; ++k) tmem_ld32(t_row + C::TMEM_S + sb * NT + 32 * k, sr + 32 * k);
+        const int col0 = half * HALF;
+        const int n_mine = min(max(n_valid - col0, 0), HALF);  // valid columns in this half
+        uint32_t sr[HALF];
+        tmem_load<HALF>(t_row + C::TMEM_S + sb * NT + col0, sr);
         tmem_ld_wait();
-        // scores in log2 units, masked past the sequence end (kept in the same registers)
-        float mt = -INFINITY;
+        // tile max of the raw scores (4 independent chains), masked past the sequence end
+        float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+        if (n_mine == HALF) {
 #pragma unroll
-        for (int k = 0; k < NT; ++k) {
-          const float xk = (k < n_valid) ? __uint_as_float(sr[k]) * sl2 : -INFINITY;
-          sr[k] = __float_as_uint(xk);
-          mt = fmaxf(mt, xk);
+          for (int k = 0; k < HALF; ++k) mx[k & 3] = fmaxf(mx[k & 3], __uint_as_float(sr[k]));
+        } else {
+#pragma unroll
+          for (int k = 0; k < HALF; ++k) {
+            if (k >= n_mine) sr[k] = __float_as_uint(-INFINITY);
+            mx[k & 3] = fmaxf(mx[k & 3], __uint_as_float(sr[k]));
+          }
         }
+        // both halves of the row agree on the tile max
+        const int rb = it & 1;
+        red_max[(rb * 2 + half) * 128 + row] = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
+        mbar_arrive(&red_bar[rb]);
+        if (!warp_wait(&red_bar[rb], (it >> 1) & 1, limit, abort_flag, status, 33)) { ok = false; break; }
+        const float mt_raw = fmaxf(red_max[(rb * 2) * 128 + row], red_max[(rb * 2 + 1) * 128 + row]);
+        const float mt = mt_raw * sl2;  // scale > 0 commutes with max
         const bool first = (j == j0);
         float factor = 1.f;
         bool rescale = false;
@@ -369,34 +412,32 @@ decode_kernel(const __grid_constant__ CUtensorMap map_ckv, const __grid_constant
           m_ref = mt;
           rescale = true;
         }
-        float sum = 0.f;
+        const float neg_m = -m_ref;
+        float sum[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-        for (int k0 = 0; k0 < NT; k0 += kPChunk) {
-          // packed fp16 pairs overwrite score registers that are already consumed
-#pragma unroll
-          for (int k = 0; k < kPChunk / 2; ++k) {
-            const float p0 = ex2_approx(__uint_as_float(sr[k0 + 2 * k]) - m_ref);
-            const float p1 = ex2_approx(__uint_as_float(sr[k0 + 2 * k + 1]) - m_ref);
-            sum += p0 + p1;
-            sr[k0 / 2 + k] = pack_f16x2(p0, p1);
-          }
-          if constexpr (kPChunk == 64) tmem_st32(t_row + C::TMEM_S + sb * NT + k0 / 2, sr + k0 / 2);
-          else tmem_st16(t_row + C::TMEM_S + sb * NT + k0 / 2, sr + k0 / 2);
+        for (int k = 0; k < HALF / 2; ++k) {
+          const float p0 = ex2_approx(fmaf(__uint_as_float(sr[2 * k]), sl2, neg_m));
+          const float p1 = ex2_approx(fmaf(__uint_as_float(sr[2 * k + 1]), sl2, neg_m));
+          sum[k & 3] += p0 + p1;
+          sr[k] = pack_f16x2(p0, p1);  // overwrites score registers already consumed
         }
-        l = first ? sum : l * factor + sum;
+        tmem_store<HALF / 2>(t_row + C::TMEM_S + sb * NT + col0 / 2, sr);
+        const float tsum = (sum[0] + sum[1]) + (sum[2] + sum[3]);
+        l = first ? tsum : fmaf(l, factor, tsum);
         if (!first) {
           // O may only be touched once the previous tile's P*V has landed.
           if (!warp_wait(pv_done, (it - 1) & 1, limit, abort_flag, status, 31)) { ok = false; break; }
           tc_fence_after();
-          if (__any_sync(0xffffffffu, rescale)) {
+          if (__any_sync(kFull, rescale)) {
 #pragma unroll 1
-            for (int k = 0; k < 4; ++k) {
+            for (int k = 0; k < 2; ++k) {
               uint32_t o[32];
-              tmem_ld32(t_row + C::TMEM_O + 32 * k, o);
+              const uint32_t oaddr = t_row + C::TMEM_O + 64 * half + 32 * k;
+              tmem_ld32(oaddr, o);
               tmem_ld_wait();
 #pragma unroll
               for (int u = 0; u < 32; ++u) o[u] = __float_as_uint(__uint_as_float(o[u]) * factor);
-              tmem_st32(t_row + C::TMEM_O + 32 * k, o);
+              tmem_st32(oaddr, o);
             }
           }
         }
@@ -409,11 +450,11 @@ decode_kernel(const __grid_constant__ CUtensorMap map_ckv, const __grid_constant
       if (!warp_wait(pv_done, (it - 1) & 1, limit, abort_flag, status, 32)) { ok = false; break; }
       tc_fence_after();
       const long long slot = static_cast<long long>(g) + s;
-      float4* dst = reinterpret_cast<float4*>(a.o_part + ((slot * 4 + slice) * 128 + row) * 128);
+      float4* dst = reinterpret_cast<float4*>(a.o_part + ((slot * 4 + slice) * 128 + row) * 128 + 64 * half);
 #pragma unroll 1
-      for (int k = 0; k < 4; ++k) {
+      for (int k = 0; k < 2; ++k) {
         uint32_t o[32];
-        tmem_ld32(t_row + C::TMEM_O + 32 * k, o);
+        tmem_ld32(t_row + C::TMEM_O + 64 * half + 32 * k, o);
         tmem_ld_wait();
         if (row < a.heads) {
 #pragma unroll
@@ -422,14 +463,20 @@ decode_kernel(const __grid_constant__ CUtensorMap map_ckv, const __grid_constant
                                          __uint_as_float(o[4 * u + 2]), __uint_as_float(o[4 * u + 3]));
         }
       }
-      if (row < a.heads) a.ml_part[(slot * 4 + slice) * 128 + row] = make_float2(m_ref, l);
+      // the row sum is split across the halves: add them once per segment
+      red_l[half * 128 + row] = l;
+      mbar_arrive(lsum_bar);
+      if (!warp_wait(lsum_bar, seg & 1, limit, abort_flag, status, 34)) { ok = false; break; }
+      ++seg;
+      if (half == 0 && row < a.heads)
+        a.ml_part[(slot * 4 + slice) * 128 + row] = make_float2(m_ref, l + red_l[128 + row]);
       tc_fence_before();
     }
   }
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 9) {
+  if (warp == 13) {
     tc_fence_after();
     tmem_dealloc(tmem, C::TMEM_COLS);
   }
@@ -448,12 +495,12 @@ cudaError_t launch_decode(const CUtensorMap& map_ckv, const CUtensorMap& map_kro
 
 }  // namespace
 
-int decode_tile_tokens(int n_branch) { return n_branch == 4 ? 128 : (n_branch == 2 ? 64 : 32); }
+int decode_tile_tokens(int n_branch) { return n_branch == 4 ? decode_split_tile_tokens() : (n_branch == 2 ? 64 : 32); }
 
 cudaError_t launch_decode_kernel(int n_branch, const CUtensorMap& map_ckv, const CUtensorMap& map_krope,
                                  const DecodeArgs& a, int groups, cudaStream_t stream) {
   switch (n_branch) {
-    case 4: return launch_decode<4, 128, 4>(map_ckv, map_krope, a, groups, stream);
+    case 4: return launch_decode_split_kernel(map_ckv, map_krope, a, groups, stream);
     case 2: return launch_decode<2, 64, 5>(map_ckv, map_krope, a, groups, stream);
     case 1: return launch_decode<1, 32, 5>(map_ckv, map_krope, a, groups, stream);
     default: return cudaErrorInvalidValue;

@@ -10,7 +10,9 @@ namespace hra {
 
 // Arguments of one decode launch (device pointers; see hra.h for layouts).
 struct DecodeArgs {
-  const __half* q_tilde;      // fp16 [B, h, 576]: absorbed latent query (512) | rotated rope (64)
+  const __half* q_tilde;      // absorbed latent query (512) | rotated rope (64) per (sequence, head):
+                              //   fp16 [B, h, 576], or for the MLRA-4 kernel bf16 hi [B, h, 576]
+                              //   followed by bf16 lo [B, h, 576]
   const int32_t* seq_lens;    // int32 [B]
   const int32_t* block_table; // int32 [B, max_pages] or nullptr (contiguous layout)
   int max_pages;
@@ -28,6 +30,11 @@ struct DecodeArgs {
 
 // Tokens per cache tile for a branch count (decides the TMEM and shared-memory budget).
 int decode_tile_tokens(int n_branch);
+int decode_split_tile_tokens();
+
+// MLRA-4 kernel on the bf16 cache with a two-term bf16 query (grid: 4 branches x groups).
+cudaError_t launch_decode_split_kernel(const CUtensorMap& map_ckv, const CUtensorMap& map_krope,
+                                       const DecodeArgs& a, int groups, cudaStream_t stream);
 
 // Launch the decode kernel on grid (4 slices, `groups` KV splits).
 cudaError_t launch_decode_kernel(int n_branch, const CUtensorMap& map_ckv, const CUtensorMap& map_krope,

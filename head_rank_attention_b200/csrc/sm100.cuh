@@ -62,6 +62,19 @@ __device__ __forceinline__ uint64_t global_ns() {
   return t;
 }
 
+// Non-blocking test of phase `parity` of `bar`.
+__device__ __forceinline__ bool mbar_test(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}\n"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
 // Bounded wait on phase `parity` of `bar`.  Gives up once `limit_ns` nanoseconds of
 // global time have passed, or as soon as another thread of the CTA has raised `*abort`;
 // on giving up it raises `*abort`, records the failure in the global status word and
@@ -150,6 +163,10 @@ __host__ __device__ constexpr uint32_t idesc_f16_f32(int M, int N, bool b_mn_maj
          | (static_cast<uint32_t>(N >> 3) << 17)      // N / 8
          | (static_cast<uint32_t>(M >> 4) << 24);     // M / 16
 }
+// Same with bf16 A/B.
+__host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, bool b_mn_major) {
+  return idesc_f16_f32(M, N, b_mn_major) | (1u << 7) | (1u << 10);
+}
 
 // D[tmem] (+)= A[tmem] * B[smem], issued by one thread.
 __device__ __forceinline__ void umma_f16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
@@ -201,6 +218,45 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t* r) {
       "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
       : "memory");
 }
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t* r) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr));
+}
+__device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t* r) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"r"(taddr), "r"(r[0]),
+               "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7])
+               : "memory");
+}
+// N consecutive 32-bit TMEM columns of this warp's 32 lanes <-> registers (N a multiple of 16 / 8).
+template <int N>
+__device__ __forceinline__ void tmem_load(uint32_t taddr, uint32_t* r) {
+  static_assert(N % 16 == 0, "tmem_load width");
+  if constexpr (N % 32 == 0) {
+#pragma unroll
+    for (int k = 0; k < N / 32; ++k) tmem_ld32(taddr + 32 * k, r + 32 * k);
+  } else {
+#pragma unroll
+    for (int k = 0; k < N / 16; ++k) tmem_ld16(taddr + 16 * k, r + 16 * k);
+  }
+}
+template <int N>
+__device__ __forceinline__ void tmem_store(uint32_t taddr, const uint32_t* r) {
+  static_assert(N % 8 == 0, "tmem_store width");
+  if constexpr (N % 32 == 0) {
+#pragma unroll
+    for (int k = 0; k < N / 32; ++k) tmem_st32(taddr + 32 * k, r + 32 * k);
+  } else if constexpr (N % 16 == 0) {
+#pragma unroll
+    for (int k = 0; k < N / 16; ++k) tmem_st16(taddr + 16 * k, r + 16 * k);
+  } else {
+#pragma unroll
+    for (int k = 0; k < N / 8; ++k) tmem_st8(taddr + 8 * k, r + 8 * k);
+  }
+}
 __device__ __forceinline__ void tmem_ld_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 __device__ __forceinline__ void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
@@ -216,6 +272,11 @@ __device__ __forceinline__ uint32_t bf16x2_to_f16x2(uint32_t v) {
   const float hi = __uint_as_float(v & 0xFFFF0000u);
   uint32_t r;
   asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  uint32_t r;
+  asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
   return r;
 }
 __device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {

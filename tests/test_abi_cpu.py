@@ -71,7 +71,7 @@ def test_workspace_size_formula():
     n = hra.workspace_size(p)
     slots = 37 + 2
     expect = 256
-    expect = -(-(expect + 2 * 128 * 576 * 2) // 256) * 256
+    expect = -(-(expect + 2 * 2 * 128 * 576 * 2) // 256) * 256  # q~ as up to two 16-bit terms
     expect = -(-(expect + slots * 4 * 128 * 128 * 4) // 256) * 256
     expect = -(-(expect + slots * 4 * 128 * 8) // 256) * 256
     assert n == expect
