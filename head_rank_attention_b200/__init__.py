@@ -7,8 +7,10 @@ supplies device memory and streams.  Build the library with
 """
 from ._binding import (EXPORTS, HRA_BF16, HRA_F32, HraDecodeParams, HraError, LIB_PATH, alloc_workspace,
                        check_device_status, last_error, load_library, make_params, mla_decode, mlra_decode,
+                       mlra_decode_static,
                        selftest_wait_timeout, version, workspace_size)
 
 __all__ = ["EXPORTS", "HRA_BF16", "HRA_F32", "HraDecodeParams", "HraError", "LIB_PATH", "alloc_workspace",
            "check_device_status", "last_error", "load_library", "make_params", "mla_decode", "mlra_decode",
+           "mlra_decode_static",
            "selftest_wait_timeout", "version", "workspace_size"]

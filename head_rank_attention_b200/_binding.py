@@ -24,7 +24,7 @@ STATUS_NAMES = {0: "HRA_OK", -1: "HRA_ERR_INVALID_ARG", -2: "HRA_ERR_UNSUPPORTED
                 -4: "HRA_ERR_CUDA", -5: "HRA_ERR_DEVICE_TIMEOUT"}
 
 # Symbols declared in include/hra.h.
-EXPORTS = ("hra_workspace_size", "mlra_decode", "mla_decode", "hra_check_device_status",
+EXPORTS = ("hra_workspace_size", "mlra_decode", "mla_decode", "mlra_decode_static", "hra_check_device_status",
            "hra_selftest_wait_timeout", "hra_last_error", "hra_version")
 
 
@@ -67,7 +67,7 @@ def load_library() -> ctypes.CDLL:
     P = ctypes.POINTER(HraDecodeParams)
     lib.hra_workspace_size.argtypes = [P]
     lib.hra_workspace_size.restype = ctypes.c_size_t
-    for name in ("mlra_decode", "mla_decode", "hra_check_device_status"):
+    for name in ("mlra_decode", "mla_decode", "mlra_decode_static", "hra_check_device_status"):
         getattr(lib, name).argtypes = [P, ctypes.c_void_p]
         getattr(lib, name).restype = ctypes.c_int
     lib.hra_selftest_wait_timeout.argtypes = [ctypes.c_void_p, ctypes.c_int, ctypes.c_void_p]
@@ -152,6 +152,12 @@ def mlra_decode(p: HraDecodeParams, stream=None) -> None:
 
 def mla_decode(p: HraDecodeParams, stream=None) -> None:
     _check(load_library().mla_decode(ctypes.byref(p), ctypes.c_void_p(_stream_handle(stream))))
+
+
+def mlra_decode_static(p: HraDecodeParams, stream=None) -> None:
+    """Decode without a workspace (scratch from the library's 32 MiB static device array):
+    for callers that cannot allocate device memory.  p.workspace is ignored."""
+    _check(load_library().mlra_decode_static(ctypes.byref(p), ctypes.c_void_p(_stream_handle(stream))))
 
 
 def check_device_status(p: HraDecodeParams, stream=None) -> None:

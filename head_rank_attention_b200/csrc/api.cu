@@ -249,6 +249,11 @@ __global__ void wait_timeout_selftest_kernel(int* status, uint64_t limit_ns) {
 
 }  // namespace
 
+namespace hra {
+// Lets other entry points of this library report through hra_last_error().
+void set_last_error(const char* msg) { g_last_error = msg; }
+}  // namespace hra
+
 extern "C" {
 
 size_t hra_workspace_size(const hra_decode_params* p) {

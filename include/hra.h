@@ -115,6 +115,19 @@ HRA_API hra_status mlra_decode(const hra_decode_params* p, void* stream /* cudaS
  * Multi-Head Latent Attention; "vllbc02MLA", decode uses the absorbed MQA-like form). */
 HRA_API hra_status mla_decode(const hra_decode_params* p, void* stream /* cudaStream_t */);
 
+/* The same decode without a caller workspace, for callers that cannot allocate device
+ * memory (code running inside another runtime's memory pool or an allocation-free
+ * serving path, plain C callers without an allocator).  The paper has no counterpart:
+ * this is a deployment variant of mlra_decode.  Scratch comes from one 32 MiB
+ * file-scope device array that every GPU loading the library holds until exit;
+ * p->workspace and p->workspace_bytes are ignored.  Calls whose hra_workspace_size
+ * exceeds 32 MiB return HRA_ERR_WORKSPACE before any CUDA call.  The first call on a
+ * device looks the array's device address up (make it before any stream capture).
+ * All calls on a device share the array: calls that overlap on the GPU race; the
+ * status word is cleared by every call, and expired device waits recorded there are
+ * not reachable through hra_check_device_status.  Allocates nothing. */
+HRA_API hra_status mlra_decode_static(const hra_decode_params* p, void* stream /* cudaStream_t */);
+
 /* Synchronize `stream` and read the device status word of p->workspace.
  * HRA_OK, or HRA_ERR_DEVICE_TIMEOUT if a bounded wait expired during the last call. */
 HRA_API hra_status hra_check_device_status(const hra_decode_params* p, void* stream);
