@@ -38,8 +38,9 @@ import synth  # noqa: E402
 METRIC = "MLRA-4 decode µs/step & KV-cache read TB/s (fraction of ~8 TB/s HBM)"
 NOMINAL_HBM_GBS = 8000.0
 FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0}
-DECODE_SOURCES = ["head_rank_attention_b200/csrc/decode_sm100.cu", "head_rank_attention_b200/csrc/sm100.cuh",
-                  "head_rank_attention_b200/csrc/schedule.cuh", "head_rank_attention_b200/csrc/decode_sm100.h"]
+DECODE_SOURCES = ["head_rank_attention_b200/csrc/decode_split_sm100.cu", "head_rank_attention_b200/csrc/decode_sm100.cu",
+                  "head_rank_attention_b200/csrc/sm100.cuh", "head_rank_attention_b200/csrc/schedule.cuh",
+                  "head_rank_attention_b200/csrc/decode_sm100.h"]
 
 
 def tensor_flops_per_token(n_branch: int, heads: int) -> int:
@@ -306,7 +307,7 @@ def run_native(args, wl, world, rank, local):
             "kv_frac_of_nominal_8TBs": kv / (step_ms * 1e-3) / 1e9 / NOMINAL_HBM_GBS,
             "stage_us": {"absorb_q": float(stage_ms[:, 0].mean()) * 1e3, "decode": decode_ms * 1e3,
                          "combine_upproj": float(stage_ms[:, 2].mean()) * 1e3},
-            "roofline": {"kernel": "decode_kernel (split-KV tcgen05)", "bound": "hbm", "achieved": achieved_gbs,
+            "roofline": {"kernel": "decode_split_kernel" if wl.n_branch == 4 else "decode_kernel", "bound": "hbm", "achieved": achieved_gbs,
                          "peak": pk["hbm_gbs"], "unit": "GB/s", "frac": achieved_gbs / pk["hbm_gbs"],
                          "peak_source": pk_src, "traffic": traffic,
                          "bytes_per_launch": kv},
