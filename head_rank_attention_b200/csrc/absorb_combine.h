@@ -2,6 +2,7 @@
 #pragma once
 
 #include <cstdint>
+#include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
@@ -10,11 +11,12 @@ namespace hra {
 
 struct AbsorbArgs {
   const __nv_bfloat16* q;     // [B, h, 192]
-  const __nv_bfloat16* w_uk;  // [h, 512, 128]
   const int32_t* seq_lens;    // [B]
   __half* q_tilde;            // out: fp16 [B, h, 576], or (two_term) bf16 hi [B, h, 576] + bf16 lo [B, h, 576]
   int two_term;               // 1: store q~ as bf16 hi + bf16 lo (MLRA-4 kernel); 0: fp16
   int* status;                // cleared by this kernel (first kernel of a call)
+  int* tile_prefix;           // out: [B + 1] exclusive prefix of decode tiles per sequence
+  int tile_tokens;            // decode tile size (tokens)
   int batch, heads;
   float alpha_q, alpha_kv, rope_theta;
 };
@@ -22,15 +24,27 @@ struct AbsorbArgs {
 struct CombineArgs {
   const float* o_part;        // [slots, 4, 128, 128]
   const float2* ml_part;      // [slots, 4, 128]
-  const int32_t* seq_lens;    // [B]
-  const __nv_bfloat16* w_uv;  // [h, 512, 128]
+  const int* tile_prefix;     // [B + 1], written by the absorb kernel
+  __nv_bfloat16* o_lat;       // merged latent output, bf16 hi [h, B, 512] then bf16 lo [h, B, 512]
+  int* status;                // device status word (expired waits)
   float* out_f32;             // [B, h, 128] or nullptr
   __nv_bfloat16* out_bf16;    // [B, h, 128] or nullptr
-  int batch, heads, groups, tile_tokens;
+  int batch, heads, groups;
   float alpha_kv, branch_scale;
 };
 
-cudaError_t launch_absorb_q(const AbsorbArgs& a, cudaStream_t stream);
-cudaError_t launch_combine_upproj(const CombineArgs& a, cudaStream_t stream);
+// Sequences per absorb CTA (the MMA's N); the q tensor map's box is {64, this} rows.
+int absorb_seq_chunk(int batch);
+// Sequences per up-projection CTA; the o_lat tensor map's box is {64, this} rows.
+int upproj_seq_chunk();
+
+// map_wuk: W_UK viewed as [h*512 rows, 128] bf16, box {64, 128}, SWIZZLE_128B.
+// map_q:   q viewed as [B rows, h*192] bf16, box {64, absorb_seq_chunk(B)}, SWIZZLE_128B.
+cudaError_t launch_absorb_q(const CUtensorMap& map_wuk, const CUtensorMap& map_q, const AbsorbArgs& a,
+                            cudaStream_t stream);
+// map_wuv:  W_UV viewed as [h*512 rows, 128] bf16, box {64, 128}, SWIZZLE_128B.
+// map_olat: a.o_lat viewed as [2*h*B rows, 512] bf16, box {64, upproj_seq_chunk()}, SWIZZLE_128B.
+cudaError_t launch_combine_upproj(const CUtensorMap& map_wuv, const CUtensorMap& map_olat, const CombineArgs& a,
+                                  cudaStream_t stream);
 
 }  // namespace hra

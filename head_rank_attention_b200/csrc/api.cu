@@ -45,7 +45,7 @@ size_t round256(size_t x) { return (x + 255) & ~size_t(255); }
 struct Plan {
   int groups = 0;
   long long slots = 0;
-  size_t q_tilde = 0, o_part = 0, ml_part = 0, total = 0;
+  size_t q_tilde = 0, o_part = 0, ml_part = 0, o_lat = 0, tile_prefix = 0, total = 0;
 };
 
 hra_status sm_count(int* n) {
@@ -117,6 +117,10 @@ hra_status make_plan(const hra_decode_params* p, Plan* plan) {
   off = round256(off + static_cast<size_t>(plan->slots) * 4 * 128 * 128 * sizeof(float));
   plan->ml_part = off;
   off = round256(off + static_cast<size_t>(plan->slots) * 4 * 128 * sizeof(float2));
+  plan->o_lat = off;  // merged latent output as two bf16 terms
+  off = round256(off + 2 * static_cast<size_t>(p->num_heads) * p->batch * 512 * sizeof(__nv_bfloat16));
+  plan->tile_prefix = off;  // decode tiles per sequence, exclusive prefix [B + 1]
+  off = round256(off + (static_cast<size_t>(p->batch) + 1) * sizeof(int));
   plan->total = off;
   return HRA_OK;
 }
@@ -124,7 +128,9 @@ hra_status make_plan(const hra_decode_params* p, Plan* plan) {
 std::once_flag g_encode_once;
 PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
 
-hra_status encode_map(CUtensorMap* map, const void* base, int64_t inner, int64_t rows, int64_t stride_elems) {
+// 2-D bf16 view [rows, inner] with row stride `stride_elems`, boxes of 64 x box_rows, 128-byte swizzle.
+hra_status encode_map(CUtensorMap* map, const void* base, int64_t inner, int64_t rows, int64_t stride_elems,
+                      int box_rows) {
   std::call_once(g_encode_once, [] {
     void* fn = nullptr;
     cudaDriverEntryPointQueryResult q{};
@@ -135,7 +141,7 @@ hra_status encode_map(CUtensorMap* map, const void* base, int64_t inner, int64_t
   if (g_encode == nullptr) return fail(HRA_ERR_CUDA, "cuTensorMapEncodeTiled entry point unavailable");
   const cuuint64_t dims[2] = {static_cast<cuuint64_t>(inner), static_cast<cuuint64_t>(rows)};
   const cuuint64_t strides[1] = {static_cast<cuuint64_t>(stride_elems) * 2};
-  const cuuint32_t box[2] = {64, 32};
+  const cuuint32_t box[2] = {64, static_cast<cuuint32_t>(box_rows)};
   const cuuint32_t estr[2] = {1, 1};
   CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -161,6 +167,23 @@ hra_status run_decode(const hra_decode_params* p, cudaStream_t stream) {
   __half* q_tilde = reinterpret_cast<__half*>(ws + plan.q_tilde);
   float* o_part = reinterpret_cast<float*>(ws + plan.o_part);
   float2* ml_part = reinterpret_cast<float2*>(ws + plan.ml_part);
+  __nv_bfloat16* o_lat = reinterpret_cast<__nv_bfloat16*>(ws + plan.o_lat);
+  int* tile_prefix = reinterpret_cast<int*>(ws + plan.tile_prefix);
+
+  // Every tensor map is encoded before the first launch so that no host work sits between
+  // the kernels of one call.
+  const int h = p->num_heads, B = p->batch;
+  CUtensorMap map_wuk, map_q, map_wuv, map_olat, map_ckv, map_krope;
+  if ((st = encode_map(&map_wuk, p->w_uk, 128, static_cast<int64_t>(h) * 512, 128, 128)) != HRA_OK) return st;
+  if ((st = encode_map(&map_q, p->q, static_cast<int64_t>(h) * 192, B, static_cast<int64_t>(h) * 192,
+                       hra::absorb_seq_chunk(B))) != HRA_OK)
+    return st;
+  if ((st = encode_map(&map_wuv, p->w_uv, 128, static_cast<int64_t>(h) * 512, 128, 128)) != HRA_OK) return st;
+  if ((st = encode_map(&map_olat, o_lat, 512, 2 * static_cast<int64_t>(h) * B, 512, hra::upproj_seq_chunk())) !=
+      HRA_OK)
+    return st;
+  if ((st = encode_map(&map_ckv, p->ckv, 512, p->cache_rows, p->ckv_stride, 32)) != HRA_OK) return st;
+  if ((st = encode_map(&map_krope, p->krope, 64, p->cache_rows, p->krope_stride, 32)) != HRA_OK) return st;
 
   auto mark = [&](int k) -> cudaError_t {
     return p->stage_events ? cudaEventRecord(static_cast<cudaEvent_t>(p->stage_events[k]), stream) : cudaSuccess;
@@ -170,7 +193,6 @@ hra_status run_decode(const hra_decode_params* p, cudaStream_t stream) {
 
   hra::AbsorbArgs ab{};
   ab.q = static_cast<const __nv_bfloat16*>(p->q);
-  ab.w_uk = static_cast<const __nv_bfloat16*>(p->w_uk);
   ab.seq_lens = p->seq_lens;
   ab.q_tilde = q_tilde;
   ab.status = status;
@@ -180,14 +202,10 @@ hra_status run_decode(const hra_decode_params* p, cudaStream_t stream) {
   ab.alpha_kv = p->alpha_kv;
   ab.rope_theta = p->rope_theta;
   ab.two_term = p->n_branch == 4 ? 1 : 0;
-  e = hra::launch_absorb_q(ab, stream);
+  ab.tile_prefix = tile_prefix;
+  ab.tile_tokens = hra::decode_tile_tokens(p->n_branch);
+  e = hra::launch_absorb_q(map_wuk, map_q, ab, stream);
   if (e != cudaSuccess) return cuda_fail(e, "absorb_q launch");
-
-  CUtensorMap map_ckv, map_krope;
-  st = encode_map(&map_ckv, p->ckv, 512, p->cache_rows, p->ckv_stride);
-  if (st != HRA_OK) return st;
-  st = encode_map(&map_krope, p->krope, 64, p->cache_rows, p->krope_stride);
-  if (st != HRA_OK) return st;
 
   const float tau = p->softmax_scale > 0.f ? p->softmax_scale : 1.0f / std::sqrt(192.0f);
   hra::DecodeArgs da{};
@@ -213,17 +231,17 @@ hra_status run_decode(const hra_decode_params* p, cudaStream_t stream) {
   hra::CombineArgs cb{};
   cb.o_part = o_part;
   cb.ml_part = ml_part;
-  cb.seq_lens = p->seq_lens;
-  cb.w_uv = static_cast<const __nv_bfloat16*>(p->w_uv);
+  cb.tile_prefix = tile_prefix;
+  cb.o_lat = o_lat;
+  cb.status = status;
   cb.out_f32 = p->out_dtype == HRA_F32 ? static_cast<float*>(p->out) : nullptr;
   cb.out_bf16 = p->out_dtype == HRA_BF16 ? static_cast<__nv_bfloat16*>(p->out) : nullptr;
   cb.batch = p->batch;
   cb.heads = p->num_heads;
   cb.groups = plan.groups;
-  cb.tile_tokens = hra::decode_tile_tokens(p->n_branch);
   cb.alpha_kv = p->alpha_kv;
   cb.branch_scale = p->branch_scale;
-  e = hra::launch_combine_upproj(cb, stream);
+  e = hra::launch_combine_upproj(map_wuv, map_olat, cb, stream);
   if (e != cudaSuccess) return cuda_fail(e, "combine_upproj launch");
   if ((e = mark(3)) != cudaSuccess) return cuda_fail(e, "stage event");
   g_last_error.clear();

@@ -74,16 +74,6 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, uint64
   return __all_sync(kFull, ok);
 }
 
-// Smallest sequence index s with prefix[s + 1] > t.
-__device__ __forceinline__ int first_seq(const int* prefix, int B, int t) {
-  int lo = 0, hi = B - 1;
-  while (lo < hi) {
-    const int mid = (lo + hi) >> 1;
-    if (prefix[mid + 1] > t) hi = mid; else lo = mid + 1;
-  }
-  return lo;
-}
-
 // O += P V for cache tile number `tile_it` (CTA-local count): A = P (fp16) from the S/P
 // buffer the tile used, B = this slice's 128 latent columns of the tile (MN-major).
 template <class C>
@@ -174,66 +164,64 @@ decode_kernel(const __grid_constant__ CUtensorMap map_ckv, const __grid_constant
   const int T = prefix[B];
   const int t_begin = T > 0 ? group_tile_begin(g, G, T) : 0;
   const int t_end = T > 0 ? group_tile_begin(g + 1, G, T) : 0;
-  const int s_first = (t_begin < t_end) ? first_seq(prefix, B, t_begin) : B;
+  const int s_first = (t_begin < t_end) ? seq_of_tile(prefix, B, t_begin) : B;
 
   if (warp == 12) {
     // ------------------------------------------------------------------ TMA producer
-    if (lane == 0) {
-      const uint64_t policy = l2_policy_evict_first();
-      int it = 0;
-      bool ok = true;
-      for (int s = s_first; ok && s < B && prefix[s] < t_end; ++s) {
-        const int j0 = max(t_begin, prefix[s]), j1 = min(t_end, prefix[s + 1]);
-        if (j0 >= j1) continue;  // empty sequence: no tiles, no segment
-        const int L = a.seq_lens[s];
-        for (int j = j0; j < j1; ++j, ++it) {
-          const int stage = it % STAGES;
-          if (it >= STAGES &&
-              !mbar_wait(&empty[stage], ((it / STAGES) + 1) & 1, limit, abort_flag, status, 1)) {
-            ok = false;
-            break;
-          }
+    // The CTA's tiles are the global tiles t_begin .. t_end-1 in order.  Each lane finds
+    // the cache row of one 32-row chunk of a batch of 32 / CHUNKS tiles (block-table and
+    // length loads in parallel), one batch ahead of the tiles lane 0 is issuing, so that
+    // no dependent global load sits between two tiles' copies.
+    constexpr int TPB = 32 / C::CHUNKS;
+    const int ntiles = t_end - t_begin;
+    const uint64_t policy = l2_policy_evict_first();
+    auto chunk_row = [&](int it0) {
+      const int t = t_begin + it0 + lane / C::CHUNKS;
+      if (t >= t_end) return static_cast<int>(a.cache_rows);
+      const int s = seq_of_tile(prefix, B, t);
+      return cache_chunk_row(a, s, (t - prefix[s]) * NT + 32 * (lane % C::CHUNKS));
+    };
+    int rows = chunk_row(0);
+    int issued = 0;
+    bool ok = true;
+    for (int it0 = 0; ok && it0 < ntiles; it0 += TPB) {
+      const int rows_next = chunk_row(it0 + TPB);
+      for (int k = 0; k < TPB && it0 + k < ntiles; ++k) {
+        const int it = it0 + k, stage = it % STAGES;
+        if (it >= STAGES && !warp_wait(&empty[stage], ((it / STAGES) + 1) & 1, limit, abort_flag, status, 1)) {
+          ok = false;
+          break;
+        }
+        int y[C::CHUNKS];
+#pragma unroll
+        for (int r = 0; r < C::CHUNKS; ++r) y[r] = __shfl_sync(kFull, rows, k * C::CHUNKS + r);
+        if (lane == 0) {
           mbar_arrive_expect_tx(&full[stage], C::STAGE_BYTES);
-          const int tok0 = (j - prefix[s]) * NT;
           uint8_t* dst = tiles + stage * C::STAGE_BYTES;
 #pragma unroll
           for (int r = 0; r < C::CHUNKS; ++r) {
-            const int t = tok0 + 32 * r;
-            long long row = a.cache_rows;  // out of range: TMA fills zeros
-            if (t < L) {
-              if (a.block_table == nullptr) {
-                row = static_cast<long long>(s) * a.seq_stride + t;
-              } else {
-                const int pidx = t / a.page_size;
-                if (pidx < a.max_pages) {
-                  const int page = a.block_table[static_cast<long long>(s) * a.max_pages + pidx];
-                  row = static_cast<long long>(page) * a.page_size + t % a.page_size;
-                }
-              }
-              if (row < 0 || row >= a.cache_rows) row = a.cache_rows;
-            }
-            const int y = static_cast<int>(row);
 #pragma unroll
             for (int d = 0; d < C::QK_BOXES; ++d) {
               void* box = dst + d * C::BOX_BYTES + r * 4096;
               if (d < C::QK_BOXES - 1)
-                tma_load_2d(box, &map_ckv, &full[stage], branch * C::W + 64 * d, y, policy);
+                tma_load_2d(box, &map_ckv, &full[stage], branch * C::W + 64 * d, y[r], policy);
               else
-                tma_load_2d(box, &map_krope, &full[stage], 0, y, policy);
+                tma_load_2d(box, &map_krope, &full[stage], 0, y[r], policy);
             }
           }
         }
+        __syncwarp();
+        issued = it + 1;
       }
-      // Tail: every stage handed out must come back before the CTA may exit, so that no
-      // copy or MMA still targets this CTA's shared memory.
-      for (int k = max(0, it - STAGES); k < it; ++k) {
-        if (ok) {
-          if (!mbar_wait(&empty[k % STAGES], (k / STAGES) & 1, limit, abort_flag, status, 2)) ok = false;
-        }
-        if (!ok) {  // aborted: wait (bounded, ignoring the abort flag) for the copy itself
-          volatile int never = 0;
-          mbar_wait(&full[k % STAGES], (k / STAGES) & 1, limit, &never, status, 3);
-        }
+      rows = rows_next;
+    }
+    // Tail: every stage handed out must come back before the CTA may exit, so that no
+    // copy or MMA still targets this CTA's shared memory.
+    for (int k = max(0, issued - STAGES); k < issued; ++k) {
+      if (ok && !warp_wait(&empty[k % STAGES], (k / STAGES) & 1, limit, abort_flag, status, 2)) ok = false;
+      if (!ok) {  // aborted: wait (bounded, ignoring the abort flag) for the copy itself
+        volatile int never = 0;
+        warp_wait(&full[k % STAGES], (k / STAGES) & 1, limit, &never, status, 3);
       }
     }
   } else if (warp == 13) {

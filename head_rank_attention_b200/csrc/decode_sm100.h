@@ -28,6 +28,28 @@ struct DecodeArgs {
   uint64_t wait_limit_ns;     // global-time budget of one device-side wait
 };
 
+// Cache row of the 32-row chunk that starts at token `tok` of sequence s (length L):
+// s * seq_stride + tok in the contiguous layout, or through the block table in the paged
+// one (pages hold a multiple of 32 rows, so a chunk never straddles two pages).  A chunk
+// that starts at or past the sequence end, or whose page is out of range, gets
+// `cache_rows`: a row past the tensor map, which the TMA fills with zeros.  The block
+// table is read before L is consulted so that both loads are in flight together.
+__device__ __forceinline__ int cache_chunk_row(const DecodeArgs& a, int s, int tok) {
+  long long row = a.cache_rows;
+  const int L = a.seq_lens[s];
+  if (a.block_table == nullptr) {
+    row = static_cast<long long>(s) * a.seq_stride + tok;
+  } else {
+    const int pidx = tok / a.page_size;
+    if (pidx < a.max_pages) {
+      const int page = a.block_table[static_cast<long long>(s) * a.max_pages + pidx];
+      row = static_cast<long long>(page) * a.page_size + tok % a.page_size;
+    }
+  }
+  if (tok >= L || row < 0 || row >= a.cache_rows) row = a.cache_rows;
+  return static_cast<int>(row);
+}
+
 // Tokens per cache tile for a branch count (decides the TMEM and shared-memory budget).
 int decode_tile_tokens(int n_branch);
 int decode_split_tile_tokens();

@@ -24,6 +24,16 @@ __device__ __forceinline__ int group_tile_begin(int g, int G, int T) {
   return static_cast<int>(static_cast<long long>(g) * T / G);
 }
 
+// Sequence that owns tile t (0 <= t < prefix[B]): the smallest s with prefix[s + 1] > t.
+__device__ __forceinline__ int seq_of_tile(const int* prefix, int B, int t) {
+  int lo = 0, hi = B - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi) >> 1;
+    if (prefix[mid + 1] > t) hi = mid; else lo = mid + 1;
+  }
+  return lo;
+}
+
 // Exclusive prefix of tiles per sequence into prefix[0..B] (prefix[B] = total), computed
 // by one full warp; lanes load 32 lengths at a time.
 __device__ __forceinline__ void tile_prefix_warp(const int32_t* __restrict__ seq_lens, int B, int NT,

@@ -74,6 +74,8 @@ def test_workspace_size_formula():
     expect = -(-(expect + 2 * 2 * 128 * 576 * 2) // 256) * 256  # q~ as up to two 16-bit terms
     expect = -(-(expect + slots * 4 * 128 * 128 * 4) // 256) * 256
     expect = -(-(expect + slots * 4 * 128 * 8) // 256) * 256
+    expect = -(-(expect + 2 * 128 * 2 * 512 * 2) // 256) * 256  # merged latent as two bf16 terms
+    expect = -(-(expect + (2 + 1) * 4) // 256) * 256  # tile prefix per sequence
     assert n == expect
 
 

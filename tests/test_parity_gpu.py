@@ -116,6 +116,27 @@ def test_zero_length_sequence_gives_zero_row():
     assert_parity(out[1:].cpu().numpy(), ref, "zero-length neighbour")
 
 
+@pytest.mark.parametrize("n_branch,page_size", [(4, 0), (4, 64), (2, 0), (2, 32), (1, 0), (1, 128)])
+def test_cache_rows_past_sequence_end_are_never_used(n_branch, page_size):
+    """Every physical cache row that holds no token of any sequence (the tail of a
+    sequence's stride or of its last page, unused pages) is NaN: the output must not
+    change, since tokens past L do not exist."""
+    wl = _case(f"nan_tail_{n_branch}_{page_size}", n_branch, (1, 31, 33, 127, 129, 300), page_size=page_size)
+    inp = synth.make_inputs(wl)
+    used = torch.zeros(inp.cache.shape[0], dtype=torch.bool)
+    for s in range(wl.batch):
+        L = int(inp.seq_lens[s])
+        idx = torch.arange(L)
+        if inp.block_table is None:
+            used[s * inp.seq_stride + idx] = True
+        else:
+            used[inp.block_table[s, idx // page_size].to(torch.int64) * page_size + idx % page_size] = True
+    assert not used.all()
+    inp.cache[~used] = float("nan")
+    out, _, _ = run_gpu(synth.to_device(inp), wl)
+    assert_parity(out.cpu().numpy(), oracle.decode_batch(inp, wl, form="absorbed"), wl.name)
+
+
 def test_bounded_wait_reports_timeout_and_context_survives():
     """A wait that nothing satisfies ends with HRA_ERR_DEVICE_TIMEOUT; the next call works."""
     wl = _case("timeout", 4, (200,))
