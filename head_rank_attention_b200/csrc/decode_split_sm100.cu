@@ -141,13 +141,13 @@ decode_split_kernel(const __grid_constant__ CUtensorMap map_ckv, const __grid_co
       mbar_init(&empty[i], 1);
     }
     mbar_init(s_full, 1);
-    mbar_init(s_free, 256);
-    mbar_init(p_ready, 256);
+    mbar_init(s_free, 8);
+    mbar_init(p_ready, 8);
     mbar_init(pv_done, 1);
-    mbar_init(q_ready, 256);
-    mbar_init(&red_bar[0], 256);
-    mbar_init(&red_bar[1], 256);
-    mbar_init(lsum_bar, 256);
+    mbar_init(q_ready, 8);
+    mbar_init(&red_bar[0], 8);
+    mbar_init(&red_bar[1], 8);
+    mbar_init(lsum_bar, 8);
     mbar_init(&drain[0], 1);
     mbar_init(&drain[1], 1);
     *abort_flag = 0;
@@ -329,7 +329,7 @@ decode_split_kernel(const __grid_constant__ CUtensorMap map_ckv, const __grid_co
         }
         tmem_st_wait();
         tc_fence_before();
-        mbar_arrive(q_ready);
+        warp_arrive(q_ready);
       }
       float m_ref = -INFINITY, l = 0.f;
       const int seg_j1 = cur.j1;
@@ -343,7 +343,7 @@ decode_split_kernel(const __grid_constant__ CUtensorMap map_ckv, const __grid_co
         tmem_load<HALF>(t_row + C::TMEM_S + half * HALF, sr);
         tmem_ld_wait();
         tc_fence_before();
-        mbar_arrive(s_free);  // the QK issuer may overwrite S once both halves got here
+        warp_arrive(s_free);  // the QK issuer may overwrite S once both halves got here
         float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
         if (n_mine == HALF) {
 #pragma unroll
@@ -357,7 +357,7 @@ decode_split_kernel(const __grid_constant__ CUtensorMap map_ckv, const __grid_co
         }
         const int rb = it & 1;
         red_max[(rb * 2 + half) * 128 + row] = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
-        mbar_arrive(&red_bar[rb]);
+        warp_arrive(&red_bar[rb]);
         if (!warp_wait(&red_bar[rb], (it >> 1) & 1, limit, abort_flag, status, 33)) { ok = false; break; }
         const float mt = fmaxf(red_max[(rb * 2) * 128 + row], red_max[(rb * 2 + 1) * 128 + row]) * sl2;
         float factor = 1.f;
@@ -410,7 +410,7 @@ decode_split_kernel(const __grid_constant__ CUtensorMap map_ckv, const __grid_co
         tmem_store<HALF / 2>(t_row + C::TMEM_P + half * (HALF / 2), sr);
         tmem_st_wait();
         tc_fence_before();
-        mbar_arrive(p_ready);
+        warp_arrive(p_ready);
       }
       if (!ok) break;
       if (!warp_wait(pv_done, (it - 1) & 1, limit, abort_flag, status, 32)) { ok = false; break; }
@@ -431,7 +431,7 @@ decode_split_kernel(const __grid_constant__ CUtensorMap map_ckv, const __grid_co
       }
       // the row sum is split across the halves: add them once per segment
       red_l[half * 128 + row] = l;
-      mbar_arrive(lsum_bar);
+      warp_arrive(lsum_bar);
       if (!warp_wait(lsum_bar, seg & 1, limit, abort_flag, status, 34)) { ok = false; break; }
       ++seg;
       if (half == 0 && row < a.heads)
