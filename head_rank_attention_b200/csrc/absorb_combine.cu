@@ -1,30 +1,35 @@
 // absorb_combine.cu -- the steps around the split-KV decode, on the tensor cores.
 //
 // absorb ("Multi-Head Low-Rank Attention", 方法步骤详情, step 1 -- query-side weight
-// absorption), one CTA per (head i, chunk of BN sequences):
-//     q~[s,i,0:512]^T = alpha_q * alpha_kv * W_UK[i] (512x128) . q_nope[s,i]^T
-// as one tcgen05 pass: A = W_UK[i] (4 M-tiles of 128 latent rows, K = 128, K-major),
-// B = the chunk's q_nope rows (N = BN, K-major), D in TMEM.  bf16 x bf16 products are
-// exact in the fp32 accumulator, so this equals the fp32 definition up to summation
-// order.  The epilogue stores q~ as fp16, or as the two-term bf16 split used by the MLRA-4
-// kernel, and rotates q_rope at position L-1 (fp64 angles: positions reach 2^21).  The
+// absorption), one CTA per (head i, chunk of 128 sequences):
+//     q~[s,i,0:512] = alpha_q * alpha_kv * q_nope[s,i] . W_UK[i]^T        (W_UK[i]: 512 x 128)
+// as one tcgen05 pass with M = the chunk's sequences, N = 512 latent (two N = 256
+// halves), K = 128: A = the q_nope rows, B = W_UK[i] (its rows are latent indices, each
+// with 128 contiguous nope dims: K-major), D in all 512 TMEM columns.  bf16 x bf16
+// products are exact in the fp32 accumulator, so this equals the fp32 definition up to
+// summation order.  A thread of the epilogue owns one sequence and 32 consecutive latent
+// columns at a time, so q~ (fp16, or the two-term bf16 split the MLRA-4 kernel uses) is
+// written with 16-byte stores.  The same threads rotate q_rope to position L-1.  The
 // branch structure needs no special case: branch b's absorbed query is columns
 // [b*w, (b+1)*w) of the same 512-vector (W_UK^(b),(i) is the matching row block).
 //
-// merge (step 2b): one warp per (sequence, 128-wide latent slice, head) combines the
-// split-KV partial states by log-sum-exp: o = sum_g 2^(m_g - M) O_g / sum_g 2^(m_g - M) l_g,
-// and stores o_lat as bf16 hi + lo terms.
+// merge (step 2b): the split-KV partial states of a (sequence, 128-wide latent slice,
+// head) are combined by log-sum-exp, o = sum_g 2^(m_g - M) O_g / sum_g 2^(m_g - M) l_g,
+// and o_lat is stored as bf16 hi + lo terms.
 //
-// upproj (step 3), one CTA per (head i, chunk of BN sequences):
-//     out[s,i,:]^T = branch_scale * alpha_kv * W_UV[i]^T (128x512) . o_lat[s,i,:]^T
-// A = W_UV[i] read MN-major (its rows are latent indices, the 128 output columns are
-// contiguous), B = o_lat hi and lo (two MMAs per K step), D in TMEM.  The branches
-// partition the latent, so summing the per-branch up-projections is this one contraction.
+// upproj (step 3), one CTA per (head i, chunk of 128 sequences):
+//     out[s,i,:] = branch_scale * alpha_kv * o_lat[s,i,:] . W_UV[i]        (W_UV[i]: 512 x 128)
+// M = sequences, N = 128 output columns, K = 512 latent (both o_lat terms): A = o_lat
+// rows (K-major), B = W_UV[i] read MN-major (its rows are latent indices with the 128
+// output columns contiguous), streamed through two shared-memory stages in four K
+// chunks.  The branches partition the latent, so summing the per-branch up-projections
+// is this one contraction.
 #include <cstdint>
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 
 #include "absorb_combine.h"
+#include "launch.h"
 #include "schedule.cuh"
 #include "sm100.cuh"
 
@@ -35,51 +40,70 @@ namespace {
 constexpr uint64_t kWaitNs = 1000000000ull;  // 1 s bound on each wait
 
 // ---------------------------------------------------------------------------- absorb
-template <int BN>
 struct AbsorbCfg {
-  static constexpr int W_BYTES = 4 * 2 * 128 * 128;  // 4 M-tiles x 2 K-boxes of [128 rows x 128 B]
-  static constexpr int Q_BYTES = 2 * BN * 128;       // 2 K-boxes of [BN rows x 128 B]
-  static constexpr int SMEM = 1024 + W_BYTES + Q_BYTES + 64;
-  static constexpr int TMEM_COLS = 4 * BN;
+  static constexpr int Q_BYTES = 2 * 128 * 128;  // 2 K boxes of [128 sequences x 128 B]
+  static constexpr int W_BYTES = 4 * 256 * 128;  // 2 latent halves x 2 K boxes of [256 rows x 128 B]
+  static constexpr int SMEM = 1024 + Q_BYTES + W_BYTES + 32 * 8 + 64;
+  static constexpr int TMEM_COLS = 512;
+  static constexpr int THREADS = 256;
 };
 
-__device__ __forceinline__ void store_q(const AbsorbArgs& a, long long idx, float x) {
-  if (a.two_term) {  // hi = bf16(x), lo = bf16(x - hi)
+// 32 consecutive fp32 values -> q~ at dst (fp16, or bf16 hi at dst and lo at dst + lo_off).
+__device__ __forceinline__ void store_q32(const AbsorbArgs& a, long long dst, long long lo_off, const float* x) {
+  if (a.two_term) {
     __nv_bfloat16* hi = reinterpret_cast<__nv_bfloat16*>(a.q_tilde);
-    const __nv_bfloat16 h = __float2bfloat16_rn(x);
-    hi[idx] = h;
-    hi[static_cast<long long>(a.batch) * a.heads * 576 + idx] = __float2bfloat16_rn(x - __bfloat162float(h));
+#pragma unroll
+    for (int v = 0; v < 4; ++v) {
+      __align__(16) __nv_bfloat16 h8[8], l8[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        h8[u] = __float2bfloat16_rn(x[8 * v + u]);
+        l8[u] = __float2bfloat16_rn(x[8 * v + u] - __bfloat162float(h8[u]));
+      }
+      *reinterpret_cast<uint4*>(hi + dst + 8 * v) = *reinterpret_cast<const uint4*>(h8);
+      *reinterpret_cast<uint4*>(hi + lo_off + dst + 8 * v) = *reinterpret_cast<const uint4*>(l8);
+    }
   } else {
-    a.q_tilde[idx] = __float2half_rn(x);
+#pragma unroll
+    for (int v = 0; v < 4; ++v) {
+      __align__(16) __half h8[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) h8[u] = __float2half_rn(x[8 * v + u]);
+      *reinterpret_cast<uint4*>(a.q_tilde + dst + 8 * v) = *reinterpret_cast<const uint4*>(h8);
+    }
   }
 }
 
-// grid (h, ceil(B / BN)), 128 threads.
-template <int BN>
-__global__ void __launch_bounds__(128, 1)
+// grid (h, ceil(B / 128)), 256 threads.  Warp w owns the sequences of TMEM lane quadrant
+// w % 4 and latent half w / 4.
+__global__ void __launch_bounds__(AbsorbCfg::THREADS, 1)
 absorb_tc_kernel(const __grid_constant__ CUtensorMap map_wuk, const __grid_constant__ CUtensorMap map_q,
                  const AbsorbArgs a) {
-  using C = AbsorbCfg<BN>;
+  using C = AbsorbCfg;
   extern __shared__ uint8_t smem_raw[];
-  uint8_t* wbuf = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* qbuf = wbuf + C::W_BYTES;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(qbuf + C::Q_BYTES);  // [0] loads landed, [1] MMAs done
+  uint8_t* qbuf = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* wbuf = qbuf + C::Q_BYTES;
+  double* turns = reinterpret_cast<double*>(wbuf + C::W_BYTES);  // [32] rope turns per position
+  uint64_t* bars = reinterpret_cast<uint64_t*>(turns + 32);      // [0] loads landed, [1] MMAs done
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   const int i = blockIdx.x;
-  const int s0 = blockIdx.y * BN;
+  const int s0 = blockIdx.y * 128;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
-  if (blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x < 4) a.status[threadIdx.x] = 0;  // fresh per call
   if (threadIdx.x == 0) {
+    grid_dep_launch();
     mbar_init(&bars[0], 1);
     mbar_init(&bars[1], 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
-  if (warp == 0) {
+  if (warp == 1) {
     tmem_alloc(tmem_slot, C::TMEM_COLS);
     tmem_relinquish();
+  }
+  if (warp == 2) {  // rotation pair j turns by theta^(-2j/64) / (2 pi) per position, in fp64
+    turns[lane] = pow(static_cast<double>(a.rope_theta), -2.0 * lane / 64.0) * 0.15915494309189535;
   }
   tc_fence_before();
   __syncthreads();
@@ -91,74 +115,121 @@ absorb_tc_kernel(const __grid_constant__ CUtensorMap map_wuk, const __grid_const
     // __syncwarp so that no lane of this warp polls a barrier lane 0 has yet to release
     if (lane == 0) {
       const uint64_t stream_once = l2_policy_evict_first();
-      mbar_arrive_expect_tx(&bars[0], C::W_BYTES + C::Q_BYTES);
-      for (int m = 0; m < 4; ++m)
-        for (int kb = 0; kb < 2; ++kb)
-          tma_load_2d(wbuf + (m * 2 + kb) * 16384, &map_wuk, &bars[0], 64 * kb, i * 512 + 128 * m, stream_once);
+      mbar_arrive_expect_tx(&bars[0], C::Q_BYTES + C::W_BYTES);
       for (int kb = 0; kb < 2; ++kb)
-        tma_load_2d(qbuf + kb * BN * 128, &map_q, &bars[0], i * 192 + 64 * kb, s0, stream_once);
+        tma_load_2d(qbuf + kb * 16384, &map_q, &bars[0], i * 192 + 64 * kb, s0, stream_once);
+      for (int n = 0; n < 2; ++n)
+        for (int kb = 0; kb < 2; ++kb)
+          tma_load_2d(wbuf + (n * 2 + kb) * 32768, &map_wuk, &bars[0], 64 * kb, i * 512 + 256 * n, stream_once);
       if (mbar_wait(&bars[0], 0, kWaitNs, abort_flag, a.status, 40)) {
         tc_fence_after();
-        constexpr uint32_t idesc = idesc_bf16_f32(128, BN, false);
-        const uint32_t wa = smem_u32(wbuf), qa = smem_u32(qbuf);
-        for (int m = 0; m < 4; ++m) {
+        constexpr uint32_t idesc = idesc_bf16_f32(128, 256, false);
+        const uint32_t qa = smem_u32(qbuf), wa = smem_u32(wbuf);
+        for (int n = 0; n < 2; ++n) {
 #pragma unroll
           for (int ks = 0; ks < 8; ++ks) {
-            const uint64_t adesc = smem_desc_sw128(wa + (m * 2 + (ks >> 2)) * 16384 + (ks & 3) * 32, 16, 1024);
-            const uint64_t bdesc = smem_desc_sw128(qa + (ks >> 2) * BN * 128 + (ks & 3) * 32, 16, 1024);
-            umma_f16_ss(tmem + m * BN, adesc, bdesc, idesc, ks > 0 ? 1u : 0u);
+            const uint64_t adesc = smem_desc_sw128(qa + (ks >> 2) * 16384 + (ks & 3) * 32, 16, 1024);
+            const uint64_t bdesc = smem_desc_sw128(wa + (n * 2 + (ks >> 2)) * 32768 + (ks & 3) * 32, 16, 1024);
+            umma_f16_ss(tmem + 256 * n, adesc, bdesc, idesc, ks > 0 ? 1u : 0u);
           }
         }
       }
       umma_commit(&bars[1]);  // arrives once every MMA issued above (possibly none) completed
     }
     __syncwarp();
-  } else {
-    const int ns = min(BN, a.batch - s0);
-    if (warp == 1 && blockIdx.x == 0 && blockIdx.y == 0) tile_prefix_warp(a.seq_lens, a.batch, a.tile_tokens, a.tile_prefix);
+  }
+  // Everything above reads only inputs of the call; what follows writes the workspace,
+  // which the previous call's kernels read, so it waits for them.
+  grid_dep_wait();
+  if (blockIdx.x == 0 && blockIdx.y == 0) {
+    if (threadIdx.x < 4) a.status[threadIdx.x] = 0;  // fresh per call
+    if (warp == 3) tile_prefix_warp(a.seq_lens, a.batch, a.tile_tokens, a.tile_prefix);
+  }
+  const int r = 32 * (warp & 3) + lane;  // sequence within the chunk = TMEM lane
+  const int s = s0 + r;
+  const int part = warp >> 2;            // latent half [256 part, +256); rope pairs [16 part, +16)
+  const long long lo_off = static_cast<long long>(a.batch) * a.heads * 576;
+  const long long row = (static_cast<long long>(s) * a.heads + i) * 576;
+  if (s < a.batch) {
     // RoPE of the query's rope part at position L-1, while the loads and MMAs run: pair
-    // (j, j + 32) turns by pos * theta^(-2j/64) radians.  The angle is carried in turns,
-    // pos * theta^(-2j/64) / (2 pi), in fp64 (pos reaches 2^21); its fractional part is
-    // exact and is then evaluated in fp32 by sincospif.  Lane = j for every thread here.
-    const double turns = pow(static_cast<double>(a.rope_theta), -2.0 * lane / 64.0) * 0.15915494309189535;
-    for (int e = threadIdx.x - 32; e < ns * 32; e += 96) {
-      const int s = s0 + e / 32;
-      const int L = a.seq_lens[s];
-      const double x = static_cast<double>(L > 0 ? L - 1 : 0) * turns;
+    // (j, j + 32) turns by pos * theta^(-2j/64) radians.  The angle is carried in turns
+    // (fp64: pos reaches 2^21); its fractional part is exact and is then evaluated in
+    // fp32 by sincospif.
+    const int L = a.seq_lens[s];
+    const double pos = static_cast<double>(L > 0 ? L - 1 : 0);
+    const uint4* qr = reinterpret_cast<const uint4*>(a.q + (static_cast<long long>(s) * a.heads + i) * 192 + 128);
+    __align__(16) __nv_bfloat16 x1[16], x2[16];
+    *reinterpret_cast<uint4*>(x1) = qr[2 * part];
+    *reinterpret_cast<uint4*>(x1 + 8) = qr[2 * part + 1];
+    *reinterpret_cast<uint4*>(x2) = qr[4 + 2 * part];
+    *reinterpret_cast<uint4*>(x2 + 8) = qr[4 + 2 * part + 1];
+    float y1[16], y2[16];
+#pragma unroll
+    for (int u = 0; u < 16; ++u) {
+      const double x = pos * turns[16 * part + u];
       const float f = static_cast<float>(x - rint(x));  // in [-1/2, 1/2]
       float sn, cs;
       sincospif(2.f * f, &sn, &cs);
-      const __nv_bfloat16* qr = a.q + (static_cast<long long>(s) * a.heads + i) * 192 + 128;
-      const float x1 = __bfloat162float(qr[lane]), x2 = __bfloat162float(qr[lane + 32]);
-      const long long off = (static_cast<long long>(s) * a.heads + i) * 576 + 512;
-      store_q(a, off + lane, fmaf(x1, cs, -x2 * sn));
-      store_q(a, off + lane + 32, fmaf(x1, sn, x2 * cs));
+      const float a1 = __bfloat162float(x1[u]), a2 = __bfloat162float(x2[u]);
+      y1[u] = fmaf(a1, cs, -a2 * sn);
+      y2[u] = fmaf(a1, sn, a2 * cs);
+    }
+    // rotated pair halves: elements [16 part, +16) and [32 + 16 part, +16) of the rope part
+    if (a.two_term) {
+      __nv_bfloat16* hi = reinterpret_cast<__nv_bfloat16*>(a.q_tilde);
+#pragma unroll
+      for (int h2 = 0; h2 < 2; ++h2) {
+        const float* y = h2 == 0 ? y1 : y2;
+        const long long dst = row + 512 + 32 * h2 + 16 * part;
+#pragma unroll
+        for (int v = 0; v < 2; ++v) {
+          __align__(16) __nv_bfloat16 h8[8], l8[8];
+#pragma unroll
+          for (int u = 0; u < 8; ++u) {
+            h8[u] = __float2bfloat16_rn(y[8 * v + u]);
+            l8[u] = __float2bfloat16_rn(y[8 * v + u] - __bfloat162float(h8[u]));
+          }
+          *reinterpret_cast<uint4*>(hi + dst + 8 * v) = *reinterpret_cast<const uint4*>(h8);
+          *reinterpret_cast<uint4*>(hi + lo_off + dst + 8 * v) = *reinterpret_cast<const uint4*>(l8);
+        }
+      }
+    } else {
+#pragma unroll
+      for (int h2 = 0; h2 < 2; ++h2) {
+        const float* y = h2 == 0 ? y1 : y2;
+        const long long dst = row + 512 + 32 * h2 + 16 * part;
+#pragma unroll
+        for (int v = 0; v < 2; ++v) {
+          __align__(16) __half h8[8];
+#pragma unroll
+          for (int u = 0; u < 8; ++u) h8[u] = __float2half_rn(y[8 * v + u]);
+          *reinterpret_cast<uint4*>(a.q_tilde + dst + 8 * v) = *reinterpret_cast<const uint4*>(h8);
+        }
+      }
     }
   }
   const bool done = mbar_wait(&bars[1], 0, kWaitNs, abort_flag, a.status, 41);
   tc_fence_after();
   if (done && !*abort_flag) {
     const float scale = a.alpha_q * a.alpha_kv;
-    const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
-    const int ns = min(BN, a.batch - s0);
+    const uint32_t lane_base = static_cast<uint32_t>(32 * (warp & 3)) << 16;
 #pragma unroll 1
-    for (int m = 0; m < 4; ++m) {
-      const int k = 128 * m + 32 * warp + lane;  // latent index = TMEM lane of tile m
-#pragma unroll 1
-      for (int c0 = 0; c0 < ns; c0 += 32) {
-        uint32_t v[32];
-        tmem_ld32(tmem + lane_base + m * BN + c0, v);
-        tmem_ld_wait();
+    for (int c = 0; c < 8; ++c) {
+      const int k0 = 256 * part + 32 * c;
+      uint32_t v[32];
+      tmem_ld32(tmem + lane_base + k0, v);
+      tmem_ld_wait();
+      if (s < a.batch) {
+        float x[32];
 #pragma unroll
-        for (int u = 0; u < 32; ++u)
-          if (c0 + u < ns)
-            store_q(a, (static_cast<long long>(s0 + c0 + u) * a.heads + i) * 576 + k, scale * __uint_as_float(v[u]));
+        for (int u = 0; u < 32; ++u) x[u] = scale * __uint_as_float(v[u]);
+        store_q32(a, row + k0, lo_off, x);
       }
     }
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == 0) {
+  if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem, C::TMEM_COLS);
   }
@@ -175,6 +246,8 @@ __global__ void __launch_bounds__(256 * Z) merge_kernel(const CombineArgs a) {
   constexpr int HPB = 256 / TPH;    // heads per block
   constexpr int V = CPT / 4;        // float4 per thread per group
   __shared__ float xchg[Z > 1 ? 256 : 1][CPT + 2];
+  if (threadIdx.x == 0) grid_dep_launch();
+  grid_dep_wait();  // the split partials and the tile prefix come from the previous kernels
   const int t = threadIdx.x & 255, z = threadIdx.x >> 8;
   const int head = blockIdx.x * HPB + t / TPH;
   const int col = (t % TPH) * CPT;  // within the slice
@@ -270,37 +343,45 @@ __global__ void __launch_bounds__(256 * Z) merge_kernel(const CombineArgs a) {
 }
 
 // ---------------------------------------------------------------------------- upproj
-template <int BN>
 struct UpprojCfg {
-  static constexpr int W_BYTES = 4 * 2 * 128 * 128;  // 4 latent blocks x 2 output-column boxes
-  static constexpr int O_BYTES = 2 * 8 * BN * 128;   // hi + lo, 8 latent boxes of [BN rows x 128 B]
-  static constexpr int SMEM = 1024 + W_BYTES + O_BYTES + 64;
-  static constexpr int TMEM_COLS = BN < 32 ? 32 : BN;
+  static constexpr int A_BYTES = 2 * 2 * 128 * 128;  // hi, lo x 2 latent boxes of [128 sequences x 128 B]
+  static constexpr int B_BYTES = 2 * 128 * 128;      // 2 output-column boxes of [128 latent rows x 128 B]
+  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+  static constexpr int STAGES = 2;
+  static constexpr int CHUNKS = 4;                   // K chunks of 128 latent
+  static constexpr int SMEM = 1024 + STAGES * STAGE_BYTES + 64;
+  static constexpr int TMEM_COLS = 128;
+  static constexpr int THREADS = 256;
 };
 
-// grid (h, ceil(B / BN)), 128 threads.
-template <int BN>
-__global__ void __launch_bounds__(128, 1)
+// grid (h, ceil(B / 128)), 256 threads.  Warp w owns the sequences of TMEM lane quadrant
+// w % 4 and output columns [64 (w / 4), +64).
+__global__ void __launch_bounds__(UpprojCfg::THREADS, 1)
 upproj_tc_kernel(const __grid_constant__ CUtensorMap map_wuv, const __grid_constant__ CUtensorMap map_olat,
                  const CombineArgs a) {
-  using C = UpprojCfg<BN>;
+  using C = UpprojCfg;
   extern __shared__ uint8_t smem_raw[];
-  uint8_t* wbuf = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* obuf = wbuf + C::W_BYTES;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(obuf + C::O_BYTES);
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2);
+  uint8_t* stages = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(stages + C::STAGES * C::STAGE_BYTES);  // [2]
+  uint64_t* empty = full + 2;                                                       // [2]
+  uint64_t* done_bar = empty + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done_bar + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   const int i = blockIdx.x;
-  const int s0 = blockIdx.y * BN;
+  const int s0 = blockIdx.y * 128;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
   if (threadIdx.x == 0) {
-    mbar_init(&bars[0], 1);
-    mbar_init(&bars[1], 1);
+    grid_dep_launch();
+    for (int k = 0; k < 2; ++k) {
+      mbar_init(&full[k], 1);
+      mbar_init(&empty[k], 1);
+    }
+    mbar_init(done_bar, 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
-  if (warp == 0) {
+  if (warp == 1) {
     tmem_alloc(tmem_slot, C::TMEM_COLS);
     tmem_relinquish();
   }
@@ -310,59 +391,121 @@ upproj_tc_kernel(const __grid_constant__ CUtensorMap map_wuv, const __grid_const
   const uint32_t tmem = *tmem_slot;
 
   if (warp == 0) {
+    // lane 0 streams the four K chunks through two stages and issues the MMAs; the other
+    // lanes wait at the __syncwarp
     if (lane == 0) {
       const uint64_t stream_once = l2_policy_evict_first();
-      mbar_arrive_expect_tx(&bars[0], C::W_BYTES + C::O_BYTES);
-      for (int kb = 0; kb < 4; ++kb)
+      const int row_hi = i * a.batch + s0;             // this head's o_lat rows
+      const int row_lo = row_hi + a.heads * a.batch;   // the lo term, h*B rows later
+      // only the 32-row boxes that hold this chunk's sequences are loaded; the other A
+      // rows feed D rows that are never stored
+      const int nbox = min(4, (a.batch - s0 + 31) / 32);
+      auto load_w = [&](int c) {  // W_UV rows of chunk c (an input of the call) + the byte count
+        uint8_t* st = stages + (c % C::STAGES) * C::STAGE_BYTES;
+        uint64_t* bar = &full[c % C::STAGES];
+        mbar_arrive_expect_tx(bar, 4 * nbox * 4096 + C::B_BYTES);
         for (int db = 0; db < 2; ++db)
-          tma_load_2d(wbuf + (kb * 2 + db) * 16384, &map_wuv, &bars[0], 64 * db, i * 512 + 128 * kb, stream_once);
-      const int row0 = i * a.batch + s0;  // this head's o_lat rows; the lo term sits h*B rows later
-      for (int part = 0; part < 2; ++part)
-        for (int kc = 0; kc < 8; ++kc)
-          tma_load_2d(obuf + (part * 8 + kc) * BN * 128, &map_olat, &bars[0], 64 * kc, row0 + part * a.heads * a.batch,
-                      stream_once);
-      if (mbar_wait(&bars[0], 0, kWaitNs, abort_flag, a.status, 42)) {
+          tma_load_2d(st + C::A_BYTES + db * 16384, &map_wuv, bar, 64 * db, i * 512 + 128 * c, stream_once);
+      };
+      auto load_o = [&](int c) {  // o_lat rows of chunk c, written by the merge kernel
+        uint8_t* st = stages + (c % C::STAGES) * C::STAGE_BYTES;
+        uint64_t* bar = &full[c % C::STAGES];
+        for (int t = 0; t < 2; ++t)
+          for (int kb = 0; kb < 2; ++kb)
+            for (int rb = 0; rb < nbox; ++rb)
+              tma_load_2d(st + (t * 2 + kb) * 16384 + rb * 4096, &map_olat, bar, 128 * c + 64 * kb,
+                          (t ? row_lo : row_hi) + 32 * rb, stream_once);
+      };
+      auto load = [&](int c) {
+        load_w(c);
+        load_o(c);
+      };
+      load_w(0);
+      load_w(1);
+      grid_dep_wait();
+      load_o(0);
+      load_o(1);
+      int issued = 2;
+      constexpr uint32_t idesc = idesc_bf16_f32(128, 128, true);  // B (W_UV) MN-major
+      const uint32_t base = smem_u32(stages);
+      bool ok = true;
+      for (int c = 0; c < C::CHUNKS && ok; ++c) {
+        const int st = c % C::STAGES;
+        if (!mbar_wait(&full[st], (c / C::STAGES) & 1, kWaitNs, abort_flag, a.status, 42)) {
+          ok = false;
+          break;
+        }
         tc_fence_after();
-        constexpr uint32_t idesc = idesc_bf16_f32(128, BN, false) | (1u << 15);  // A MN-major
-        const uint32_t wa = smem_u32(wbuf), oa = smem_u32(obuf);
-#pragma unroll 1
-        for (int ks = 0; ks < 32; ++ks) {  // latent rows k = 16 ks .. 16 ks + 15
-          const uint64_t adesc = smem_desc_sw128(wa + (ks >> 3) * 2 * 16384 + (ks & 7) * 2048, 16384, 1024);
+        const uint32_t sa = base + st * C::STAGE_BYTES, sb = sa + C::A_BYTES;
 #pragma unroll
-          for (int part = 0; part < 2; ++part) {
-            const uint64_t bdesc = smem_desc_sw128(oa + (part * 8 + (ks >> 2)) * BN * 128 + (ks & 3) * 32, 16, 1024);
-            umma_f16_ss(tmem, adesc, bdesc, idesc, (ks > 0 || part > 0) ? 1u : 0u);
+        for (int ks = 0; ks < 8; ++ks) {  // latent rows 128 c + 16 ks .. + 15
+          const uint64_t bdesc = smem_desc_sw128(sb + ks * 2048, 16384, 1024);
+#pragma unroll
+          for (int t = 0; t < 2; ++t) {
+            const uint64_t adesc = smem_desc_sw128(sa + (t * 2 + (ks >> 2)) * 16384 + (ks & 3) * 32, 16, 1024);
+            umma_f16_ss(tmem, adesc, bdesc, idesc, (c > 0 || ks > 0 || t > 0) ? 1u : 0u);
           }
         }
+        umma_commit(&empty[st]);
+        // refill the other stage once the previous chunk's MMAs (queued ahead of these)
+        // have read it
+        if (c >= 1 && c + 1 < C::CHUNKS) {
+          const int prev = c - 1;
+          if (!mbar_wait(&empty[prev % C::STAGES], (prev / C::STAGES) & 1, kWaitNs, abort_flag, a.status, 43)) {
+            ok = false;
+            break;
+          }
+          load(c + 1);
+          ++issued;
+        }
       }
-      umma_commit(&bars[1]);
+      umma_commit(done_bar);  // every MMA issued above (possibly none) completed
+      if (!ok) {  // copies still in flight land before the CTA may exit
+        volatile int never = 0;
+        for (int k = issued - C::STAGES; k < issued; ++k)
+          mbar_wait(&full[k % C::STAGES], (k / C::STAGES) & 1, kWaitNs, &never, a.status, 44);
+      }
     }
     __syncwarp();
   }
-  const bool done = mbar_wait(&bars[1], 0, kWaitNs, abort_flag, a.status, 43);
+  grid_dep_wait();  // (a no-op after the first) before writing out and reading the status
+  const bool done = mbar_wait(done_bar, 0, kWaitNs, abort_flag, a.status, 45);
   tc_fence_after();
+  const int r = 32 * (warp & 3) + lane;  // sequence within the chunk = TMEM lane
+  const int s = s0 + r;
+  const int part = warp >> 2;
   if (done && !*abort_flag) {
     const float scale = a.branch_scale * a.alpha_kv;
-    const int d = 32 * warp + lane;  // output column = TMEM lane
-    const int ns = min(BN, a.batch - s0);
+    const uint32_t lane_base = static_cast<uint32_t>(32 * (warp & 3)) << 16;
 #pragma unroll 1
-    for (int c0 = 0; c0 < BN; c0 += 16) {
-      uint32_t v[16];
-      tmem_ld16(tmem + (static_cast<uint32_t>(warp * 32) << 16) + c0, v);
+    for (int c = 0; c < 2; ++c) {
+      const int d0 = 64 * part + 32 * c;
+      uint32_t v[32];
+      tmem_ld32(tmem + lane_base + d0, v);
       tmem_ld_wait();
+      if (s < a.batch) {
+        const long long o = (static_cast<long long>(s) * a.heads + i) * 128 + d0;
+        if (a.out_f32) {
 #pragma unroll
-      for (int u = 0; u < 16; ++u) {
-        if (c0 + u >= ns) continue;
-        const long long o = (static_cast<long long>(s0 + c0 + u) * a.heads + i) * 128 + d;
-        const float val = scale * __uint_as_float(v[u]);
-        if (a.out_f32) a.out_f32[o] = val;
-        else a.out_bf16[o] = __float2bfloat16_rn(val);
+          for (int q = 0; q < 8; ++q)
+            *reinterpret_cast<float4*>(a.out_f32 + o + 4 * q) =
+                make_float4(scale * __uint_as_float(v[4 * q]), scale * __uint_as_float(v[4 * q + 1]),
+                            scale * __uint_as_float(v[4 * q + 2]), scale * __uint_as_float(v[4 * q + 3]));
+        } else {
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            __align__(16) __nv_bfloat16 b8[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) b8[u] = __float2bfloat16_rn(scale * __uint_as_float(v[8 * q + u]));
+            *reinterpret_cast<uint4*>(a.out_bf16 + o + 8 * q) = *reinterpret_cast<const uint4*>(b8);
+          }
+        }
       }
     }
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == 0) {
+  if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem, C::TMEM_COLS);
   }
@@ -375,38 +518,30 @@ cudaError_t set_smem(K kern, int bytes) {
 
 }  // namespace
 
-int absorb_seq_chunk(int batch) { return batch <= 32 ? 32 : 128; }
+int absorb_seq_chunk(int) { return 128; }
 int upproj_seq_chunk() { return 32; }
 
 cudaError_t launch_absorb_q(const CUtensorMap& map_wuk, const CUtensorMap& map_q, const AbsorbArgs& a,
-                            cudaStream_t stream) {
-  cudaError_t e;
-  if (absorb_seq_chunk(a.batch) == 32) {
-    if ((e = set_smem(absorb_tc_kernel<32>, AbsorbCfg<32>::SMEM)) != cudaSuccess) return e;
-    absorb_tc_kernel<32><<<dim3(a.heads, (a.batch + 31) / 32), 128, AbsorbCfg<32>::SMEM, stream>>>(map_wuk, map_q, a);
-  } else {
-    if ((e = set_smem(absorb_tc_kernel<128>, AbsorbCfg<128>::SMEM)) != cudaSuccess) return e;
-    absorb_tc_kernel<128><<<dim3(a.heads, (a.batch + 127) / 128), 128, AbsorbCfg<128>::SMEM, stream>>>(map_wuk,
-                                                                                                         map_q, a);
-  }
-  return cudaGetLastError();
+                            cudaStream_t stream, bool pdl) {
+  cudaError_t e = set_smem(absorb_tc_kernel, AbsorbCfg::SMEM);
+  if (e != cudaSuccess) return e;
+  return launch_kernel(absorb_tc_kernel, dim3(a.heads, (a.batch + 127) / 128), dim3(AbsorbCfg::THREADS),
+                       AbsorbCfg::SMEM, stream, pdl, map_wuk, map_q, a);
 }
 
 cudaError_t launch_combine_upproj(const CUtensorMap& map_wuv, const CUtensorMap& map_olat, const CombineArgs& a,
-                                  cudaStream_t stream) {
+                                  cudaStream_t stream, bool pdl) {
   // Many sequences: 32 heads x 4 float4 per block.  Few sequences (each spread over many
   // groups): 8 heads x 1 float4 per block and two thread sets over alternate group runs.
+  cudaError_t e;
   if (a.batch >= 16)
-    merge_kernel<16, 1, 2><<<dim3((a.heads + 31) / 32, 4, a.batch), 256, 0, stream>>>(a);
+    e = launch_kernel(merge_kernel<16, 1, 2>, dim3((a.heads + 31) / 32, 4, a.batch), dim3(256), 0, stream, pdl, a);
   else
-    merge_kernel<4, 2, 4><<<dim3((a.heads + 7) / 8, 4, a.batch), 512, 0, stream>>>(a);
-  cudaError_t e = cudaGetLastError();
+    e = launch_kernel(merge_kernel<4, 2, 4>, dim3((a.heads + 7) / 8, 4, a.batch), dim3(512), 0, stream, pdl, a);
   if (e != cudaSuccess) return e;
-  constexpr int BN = 32;
-  if ((e = set_smem(upproj_tc_kernel<BN>, UpprojCfg<BN>::SMEM)) != cudaSuccess) return e;
-  upproj_tc_kernel<BN><<<dim3(a.heads, (a.batch + BN - 1) / BN), 128, UpprojCfg<BN>::SMEM, stream>>>(map_wuv,
-                                                                                                       map_olat, a);
-  return cudaGetLastError();
+  if ((e = set_smem(upproj_tc_kernel, UpprojCfg::SMEM)) != cudaSuccess) return e;
+  return launch_kernel(upproj_tc_kernel, dim3(a.heads, (a.batch + 127) / 128), dim3(UpprojCfg::THREADS),
+                       UpprojCfg::SMEM, stream, pdl, map_wuv, map_olat, a);
 }
 
 }  // namespace hra

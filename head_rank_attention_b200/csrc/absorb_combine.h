@@ -33,18 +33,19 @@ struct CombineArgs {
   float alpha_kv, branch_scale;
 };
 
-// Sequences per absorb CTA (the MMA's N); the q tensor map's box is {64, this} rows.
+// Sequences per absorb CTA (the MMA's M); the q tensor map's box is {64, this} rows.
 int absorb_seq_chunk(int batch);
-// Sequences per up-projection CTA; the o_lat tensor map's box is {64, this} rows.
+// Rows of one o_lat box in the up-projection (its CTAs take 128 sequences in boxes of this many).
 int upproj_seq_chunk();
 
-// map_wuk: W_UK viewed as [h*512 rows, 128] bf16, box {64, 128}, SWIZZLE_128B.
+// map_wuk: W_UK viewed as [h*512 rows, 128] bf16, box {64, 256}, SWIZZLE_128B.
 // map_q:   q viewed as [B rows, h*192] bf16, box {64, absorb_seq_chunk(B)}, SWIZZLE_128B.
+// pdl: launch with programmatic dependent launch (launch.h).
 cudaError_t launch_absorb_q(const CUtensorMap& map_wuk, const CUtensorMap& map_q, const AbsorbArgs& a,
-                            cudaStream_t stream);
+                            cudaStream_t stream, bool pdl);
 // map_wuv:  W_UV viewed as [h*512 rows, 128] bf16, box {64, 128}, SWIZZLE_128B.
 // map_olat: a.o_lat viewed as [2*h*B rows, 512] bf16, box {64, upproj_seq_chunk()}, SWIZZLE_128B.
 cudaError_t launch_combine_upproj(const CUtensorMap& map_wuv, const CUtensorMap& map_olat, const CombineArgs& a,
-                                  cudaStream_t stream);
+                                  cudaStream_t stream, bool pdl);
 
 }  // namespace hra

@@ -174,7 +174,7 @@ hra_status run_decode(const hra_decode_params* p, cudaStream_t stream) {
   // the kernels of one call.
   const int h = p->num_heads, B = p->batch;
   CUtensorMap map_wuk, map_q, map_wuv, map_olat, map_ckv, map_krope;
-  if ((st = encode_map(&map_wuk, p->w_uk, 128, static_cast<int64_t>(h) * 512, 128, 128)) != HRA_OK) return st;
+  if ((st = encode_map(&map_wuk, p->w_uk, 128, static_cast<int64_t>(h) * 512, 128, 256)) != HRA_OK) return st;
   if ((st = encode_map(&map_q, p->q, static_cast<int64_t>(h) * 192, B, static_cast<int64_t>(h) * 192,
                        hra::absorb_seq_chunk(B))) != HRA_OK)
     return st;
@@ -204,7 +204,10 @@ hra_status run_decode(const hra_decode_params* p, cudaStream_t stream) {
   ab.two_term = p->n_branch == 4 ? 1 : 0;
   ab.tile_prefix = tile_prefix;
   ab.tile_tokens = hra::decode_tile_tokens(p->n_branch);
-  e = hra::launch_absorb_q(map_wuk, map_q, ab, stream);
+  // Programmatic dependent launch lets each kernel start while the previous one drains;
+  // the stage-timing mode launches plainly so that its events bracket whole kernels.
+  const bool pdl = p->stage_events == nullptr;
+  e = hra::launch_absorb_q(map_wuk, map_q, ab, stream, pdl);
   if (e != cudaSuccess) return cuda_fail(e, "absorb_q launch");
 
   const float tau = p->softmax_scale > 0.f ? p->softmax_scale : 1.0f / std::sqrt(192.0f);
@@ -224,7 +227,7 @@ hra_status run_decode(const hra_decode_params* p, cudaStream_t stream) {
   da.status = status;
   da.wait_limit_ns = 1000ull * (p->wait_limit > 0 ? static_cast<uint64_t>(p->wait_limit) : kDefaultWaitLimitUs);
   if ((e = mark(1)) != cudaSuccess) return cuda_fail(e, "stage event");
-  e = hra::launch_decode_kernel(p->n_branch, map_ckv, map_krope, da, plan.groups, stream);
+  e = hra::launch_decode_kernel(p->n_branch, map_ckv, map_krope, da, plan.groups, stream, pdl);
   if (e != cudaSuccess) return cuda_fail(e, "decode launch");
   if ((e = mark(2)) != cudaSuccess) return cuda_fail(e, "stage event");
 
@@ -241,7 +244,7 @@ hra_status run_decode(const hra_decode_params* p, cudaStream_t stream) {
   cb.groups = plan.groups;
   cb.alpha_kv = p->alpha_kv;
   cb.branch_scale = p->branch_scale;
-  e = hra::launch_combine_upproj(map_wuv, map_olat, cb, stream);
+  e = hra::launch_combine_upproj(map_wuv, map_olat, cb, stream, pdl);
   if (e != cudaSuccess) return cuda_fail(e, "combine_upproj launch");
   if ((e = mark(3)) != cudaSuccess) return cuda_fail(e, "stage event");
   g_last_error.clear();

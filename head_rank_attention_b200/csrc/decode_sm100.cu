@@ -30,6 +30,7 @@
 #include <cstdint>
 
 #include "decode_sm100.h"
+#include "launch.h"
 #include "schedule.cuh"
 #include "sm100.cuh"
 
@@ -130,6 +131,7 @@ decode_kernel(const __grid_constant__ CUtensorMap map_ckv, const __grid_constant
   int* status = a.status;
 
   if (warp == 0) tile_prefix_warp(a.seq_lens, B, NT, prefix);
+  if (threadIdx.x == 0) grid_dep_launch();
   if (threadIdx.x == 32) {
     for (int i = 0; i < STAGES; ++i) {
       mbar_init(&full[i], 1);
@@ -327,6 +329,9 @@ decode_kernel(const __grid_constant__ CUtensorMap map_ckv, const __grid_constant
     }
   } else {
     // ------------------------------------------------------------------ softmax + epilogue
+    // The absorbed query comes from the previous kernel, and the split partials written
+    // here are read by the previous call's merge: wait for those grids.
+    grid_dep_wait();
     constexpr int HALF = C::HALF;
     const int half = warp >> 2;                        // which half of the score columns
     const int row = threadIdx.x & 127;                 // head row == TMEM lane
@@ -472,13 +477,12 @@ decode_kernel(const __grid_constant__ CUtensorMap map_ckv, const __grid_constant
 
 template <int NB, int NT, int STAGES>
 cudaError_t launch_decode(const CUtensorMap& map_ckv, const CUtensorMap& map_krope, const DecodeArgs& a,
-                          int groups, cudaStream_t stream) {
+                          int groups, cudaStream_t stream, bool pdl) {
   using C = DecodeCfg<NB, NT, STAGES>;
   auto kern = decode_kernel<NB, NT, STAGES>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
   if (e != cudaSuccess) return e;
-  kern<<<dim3(4, groups), C::THREADS, C::SMEM_BYTES, stream>>>(map_ckv, map_krope, a);
-  return cudaGetLastError();
+  return launch_kernel(kern, dim3(4, groups), dim3(C::THREADS), C::SMEM_BYTES, stream, pdl, map_ckv, map_krope, a);
 }
 
 }  // namespace
@@ -486,11 +490,11 @@ cudaError_t launch_decode(const CUtensorMap& map_ckv, const CUtensorMap& map_kro
 int decode_tile_tokens(int n_branch) { return n_branch == 4 ? decode_split_tile_tokens() : (n_branch == 2 ? 64 : 32); }
 
 cudaError_t launch_decode_kernel(int n_branch, const CUtensorMap& map_ckv, const CUtensorMap& map_krope,
-                                 const DecodeArgs& a, int groups, cudaStream_t stream) {
+                                 const DecodeArgs& a, int groups, cudaStream_t stream, bool pdl) {
   switch (n_branch) {
-    case 4: return launch_decode_split_kernel(map_ckv, map_krope, a, groups, stream);
-    case 2: return launch_decode<2, 64, 5>(map_ckv, map_krope, a, groups, stream);
-    case 1: return launch_decode<1, 32, 5>(map_ckv, map_krope, a, groups, stream);
+    case 4: return launch_decode_split_kernel(map_ckv, map_krope, a, groups, stream, pdl);
+    case 2: return launch_decode<2, 64, 5>(map_ckv, map_krope, a, groups, stream, pdl);
+    case 1: return launch_decode<1, 32, 5>(map_ckv, map_krope, a, groups, stream, pdl);
     default: return cudaErrorInvalidValue;
   }
 }

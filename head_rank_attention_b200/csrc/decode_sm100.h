@@ -56,10 +56,11 @@ int decode_split_tile_tokens();
 
 // MLRA-4 kernel on the bf16 cache with a two-term bf16 query (grid: 4 branches x groups).
 cudaError_t launch_decode_split_kernel(const CUtensorMap& map_ckv, const CUtensorMap& map_krope,
-                                       const DecodeArgs& a, int groups, cudaStream_t stream);
+                                       const DecodeArgs& a, int groups, cudaStream_t stream, bool pdl);
 
-// Launch the decode kernel on grid (4 slices, `groups` KV splits).
+// Launch the decode kernel on grid (4 slices, `groups` KV splits); pdl: programmatic
+// dependent launch (launch.h).
 cudaError_t launch_decode_kernel(int n_branch, const CUtensorMap& map_ckv, const CUtensorMap& map_krope,
-                                 const DecodeArgs& a, int groups, cudaStream_t stream);
+                                 const DecodeArgs& a, int groups, cudaStream_t stream, bool pdl);
 
 }  // namespace hra

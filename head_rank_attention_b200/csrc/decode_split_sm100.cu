@@ -25,6 +25,7 @@
 #include <cstdint>
 
 #include "decode_sm100.h"
+#include "launch.h"
 #include "schedule.cuh"
 #include "sm100.cuh"
 
@@ -135,6 +136,7 @@ decode_split_kernel(const __grid_constant__ CUtensorMap map_ckv, const __grid_co
   int* status = a.status;
 
   if (warp == 0) tile_prefix_warp(a.seq_lens, B, NT, prefix);
+  if (threadIdx.x == 0) grid_dep_launch();
   if (threadIdx.x == 32) {
     for (int i = 0; i < STAGES; ++i) {
       mbar_init(&full[i], 1);
@@ -296,6 +298,10 @@ decode_split_kernel(const __grid_constant__ CUtensorMap map_ckv, const __grid_co
     }
   } else if (warp < 8) {
     // ------------------------------------------------------------------ softmax + epilogue
+    // The absorbed query comes from the previous kernel, and the split partials written
+    // here are read by the previous call's merge: wait for those grids.  The producer and
+    // the MMA issuers touch no memory another kernel writes.
+    grid_dep_wait();
     const int half = warp >> 2;           // score columns [half*HALF, +HALF), O columns [64 half, +64)
     const int row = threadIdx.x & 127;    // head row == TMEM lane
     const uint32_t t_row = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
@@ -453,13 +459,12 @@ decode_split_kernel(const __grid_constant__ CUtensorMap map_ckv, const __grid_co
 int decode_split_tile_tokens() { return kNT; }
 
 cudaError_t launch_decode_split_kernel(const CUtensorMap& map_ckv, const CUtensorMap& map_krope,
-                                       const DecodeArgs& a, int groups, cudaStream_t stream) {
+                                       const DecodeArgs& a, int groups, cudaStream_t stream, bool pdl) {
   using C = SplitCfg<kNT, kStages>;
   auto kern = decode_split_kernel<kNT, kStages>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
   if (e != cudaSuccess) return e;
-  kern<<<dim3(4, groups), C::THREADS, C::SMEM_BYTES, stream>>>(map_ckv, map_krope, a);
-  return cudaGetLastError();
+  return launch_kernel(kern, dim3(4, groups), dim3(C::THREADS), C::SMEM_BYTES, stream, pdl, map_ckv, map_krope, a);
 }
 
 }  // namespace hra

@@ -1,0 +1,32 @@
+// launch.h -- kernel launches with programmatic dependent launch (PDL).
+//
+// A kernel launched with pdl = true may start while the previous kernel on the stream is
+// still running: its CTAs run their set-up (barriers, TMEM, loads of inputs no earlier
+// kernel writes) and then execute griddepcontrol.wait (grid_dep_wait in sm100.cuh), which
+// returns once the previous grid has completed and its writes are visible.  Every kernel
+// of the decode path therefore reads the outputs of earlier kernels, and writes anything
+// an earlier kernel reads, only after grid_dep_wait.  Each kernel also signals
+// griddepcontrol.launch_dependents early so that the next one can be scheduled.
+#pragma once
+
+#include <cuda_runtime.h>
+
+namespace hra {
+
+template <typename... KArgs, typename... Args>
+cudaError_t launch_kernel(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream, bool pdl,
+                          Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...);
+}
+
+}  // namespace hra

@@ -137,6 +137,28 @@ def test_cache_rows_past_sequence_end_are_never_used(n_branch, page_size):
     assert_parity(out.cpu().numpy(), oracle.decode_batch(inp, wl, form="absorbed"), wl.name)
 
 
+def test_back_to_back_calls_sharing_a_workspace():
+    """Calls queued back to back on one stream, sharing one workspace, with different
+    inputs: each call's kernels may start while the previous call drains, so any write
+    of the workspace before the previous call is done with it would change an output."""
+    wl_a = _case("b2b_a", 4, (3000, 17, 900))
+    wl_b = _case("b2b_b", 4, (40, 2500, 700), seed=7)
+    dev_a, dev_b = synth.to_device(synth.make_inputs(wl_a)), synth.to_device(synth.make_inputs(wl_b))
+    ref_a, p_a, ws = run_gpu(dev_a, wl_a)
+    ref_b, p_b, _ = run_gpu(dev_b, wl_b, workspace=ws)
+    outs = []
+    for k in range(6):
+        dev, wl, p = (dev_a, wl_a, p_a) if k % 2 == 0 else (dev_b, wl_b, p_b)
+        out = torch.empty_like(ref_a)
+        p.out = out.data_ptr()
+        hra.mlra_decode(p)
+        outs.append(out)
+    torch.cuda.synchronize()
+    hra.check_device_status(p_a)
+    for k, out in enumerate(outs):
+        assert torch.equal(out, ref_a if k % 2 == 0 else ref_b), f"call {k}"
+
+
 def test_bounded_wait_reports_timeout_and_context_survives():
     """A wait that nothing satisfies ends with HRA_ERR_DEVICE_TIMEOUT; the next call works."""
     wl = _case("timeout", 4, (200,))
