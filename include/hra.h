@@ -22,9 +22,14 @@
  * message from hra_last_error() (thread-local).  Launch failures return HRA_ERR_CUDA.
  * Bounded device waits that expire write a status word in the workspace, read back
  * by hra_check_device_status().
- * Numerics: bf16 inputs; the tensor-core contractions run on fp16 operands (the cache
- * tile is converted in shared memory, so |cache values| must stay below 65504) with
- * fp32 accumulation; softmax, combine and up-projection in fp32.
+ * Numerics: bf16 inputs, fp32 accumulation; softmax, combine and up-projection in fp32.
+ * n_branch = 4: the tensor cores read the bf16 cache as stored, against the absorbed
+ * query carried as two bf16 terms (hi + lo, ~16 significant bits).
+ * n_branch = 1, 2: the cache tile is converted to fp16 in shared memory and the query is
+ * fp16, so |cache values| must stay below 65504.
+ * Stream order: the kernels of a call are chained with programmatic dependent launch, so
+ * a call may begin (set-up, loads of its inputs) while the previous call on the stream
+ * drains; it touches the workspace only once that call has completed.
  */
 #ifndef HRA_H
 #define HRA_H
