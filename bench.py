@@ -242,18 +242,51 @@ def run_native(args, wl, world, rank, local):
             torch.distributed.barrier()
         torch.cuda.synchronize()
 
+    # Inputs smaller than twice the L2 (126 MB) would stay cached between steps: flush it
+    # by writing a 512 MB buffer before every timed step.
+    step_bytes = kv + sum(t.numel() * t.element_size() for t in (dev.q, dev.w_uk, dev.w_uv))
+    flush = torch.zeros(128 << 20, dtype=torch.float32, device="cuda") if step_bytes < (252 << 20) else None
+
     # The timed steps: the call as a user makes it (kernels chained by programmatic
-    # dependent launch).
-    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    # dependent launch), replayed from a CUDA graph of one call unless --no-graph, so that
+    # host-side launch work does not bound the short configurations.
+    graph = None
+    if not args.no_graph:
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            hra.mlra_decode(p, torch.cuda.current_stream())
+        for _ in range(args.warmup):
+            graph.replay()
+        torch.cuda.synchronize()
+        hra.check_device_status(p, stream)
+    def one_step():
+        if graph is not None:
+            graph.replay()
+        else:
+            hra.mlra_decode(p, stream)
+
     barrier()
     with ClockSampler(dev_id) as clk:
-        start.record(stream)
-        for k in range(args.steps):
-            hra.mlra_decode(p, stream)
-        end.record(stream)
-        torch.cuda.synchronize()
+        if flush is None:  # inputs larger than L2: back-to-back steps
+            start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            start.record(stream)
+            for k in range(args.steps):
+                one_step()
+            end.record(stream)
+            torch.cuda.synchronize()
+            elapsed_ms = start.elapsed_time(end)
+        else:  # small inputs: L2 flushed before every step, each step timed on its own
+            pairs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                     for _ in range(args.steps)]
+            for e0, e1 in pairs:
+                flush.add_(1)
+                e0.record(stream)
+                one_step()
+                e1.record(stream)
+            torch.cuda.synchronize()
+            elapsed_ms = sum(e0.elapsed_time(e1) for e0, e1 in pairs)
     hra.check_device_status(p, stream)
-    elapsed_ms = start.elapsed_time(end)
+    del graph
 
     # Per-stage breakdown (and the decode kernel's own time for the roofline): the same
     # number of steps again with events between the kernels, which the library then
@@ -319,7 +352,11 @@ def run_native(args, wl, world, rank, local):
                           "fp32 accumulate, softmax, combine"),
             "data": "synthetic",
             "config": dict(workload_config(wl, lens), parallelism=f"replicas x{world}" if world > 1 else "1 GPU",
-                           num_splits=args.num_splits or "auto (SMs/4)"),
+                           num_splits=args.num_splits or "auto (SMs/4)",
+                           timing="CUDA-graph replays of one call" if not args.no_graph else "direct calls",
+                           **({} if flush is None else
+                              {"l2": "inputs smaller than L2: 512 MB written before every step, "
+                                     "each step timed on its own"})),
             "kv_frac_of_nominal_8TBs": kv / (step_ms * 1e-3) / 1e9 / NOMINAL_HBM_GBS,
             "stage_us": {"absorb_q": float(stage_ms[:, 0].mean()) * 1e3, "decode": decode_ms * 1e3,
                          "combine_upproj": float(stage_ms[:, 2].mean()) * 1e3},
@@ -364,6 +401,7 @@ def main():
     ap.add_argument("--ref-seqs", type=int, default=1)
     ap.add_argument("--ref-heads", type=int, default=8)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-graph", action="store_true", help="time direct calls instead of CUDA-graph replays")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

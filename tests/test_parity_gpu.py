@@ -159,6 +159,26 @@ def test_back_to_back_calls_sharing_a_workspace():
         assert torch.equal(out, ref_a if k % 2 == 0 else ref_b), f"call {k}"
 
 
+@pytest.mark.parametrize("n_branch", [4, 1])
+def test_cuda_graph_replay_matches_direct_call(n_branch):
+    """A call captured into a CUDA graph (kernels chained programmatically inside it)
+    and replayed gives the bits of a direct call."""
+    wl = _case(f"graph_{n_branch}", n_branch, (1500, 40))
+    dev = synth.to_device(synth.make_inputs(wl))
+    ref, p, ws = run_gpu(dev, wl)
+    out = torch.zeros_like(ref)
+    p.out = out.data_ptr()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        hra.mlra_decode(p, torch.cuda.current_stream())
+    for _ in range(3):
+        out.zero_()
+        g.replay()
+        torch.cuda.synchronize()
+        assert torch.equal(out, ref)
+    hra.check_device_status(p)
+
+
 def test_bounded_wait_reports_timeout_and_context_survives():
     """A wait that nothing satisfies ends with HRA_ERR_DEVICE_TIMEOUT; the next call works."""
     wl = _case("timeout", 4, (200,))
