@@ -175,25 +175,7 @@ absorb_tc_kernel(const __grid_constant__ CUtensorMap map_wuk, const __grid_const
       y2[u] = fmaf(a1, sn, a2 * cs);
     }
     // rotated pair halves: elements [16 part, +16) and [32 + 16 part, +16) of the rope part
-    if (a.two_term) {
-      __nv_bfloat16* hi = reinterpret_cast<__nv_bfloat16*>(a.q_tilde);
-#pragma unroll
-      for (int h2 = 0; h2 < 2; ++h2) {
-        const float* y = h2 == 0 ? y1 : y2;
-        const long long dst = row + 512 + 32 * h2 + 16 * part;
-#pragma unroll
-        for (int v = 0; v < 2; ++v) {
-          __align__(16) __nv_bfloat16 h8[8], l8[8];
-#pragma unroll
-          for (int u = 0; u < 8; ++u) {
-            h8[u] = __float2bfloat16_rn(y[8 * v + u]);
-            l8[u] = __float2bfloat16_rn(y[8 * v + u] - __bfloat162float(h8[u]));
-          }
-          *reinterpret_cast<uint4*>(hi + dst + 8 * v) = *reinterpret_cast<const uint4*>(h8);
-          *reinterpret_cast<uint4*>(hi + lo_off + dst + 8 * v) = *reinterpret_cast<const uint4*>(l8);
-        }
-      }
-    } else {
+    {  // fp16 in both modes (the two-term query's rope slot of the hi array)
 #pragma unroll
       for (int h2 = 0; h2 < 2; ++h2) {
         const float* y = h2 == 0 ? y1 : y2;

@@ -3,23 +3,26 @@
 //
 // Same computation and work decomposition as decode_sm100.cu (step 2 of "Multi-Head
 // Low-Rank Attention", 方法步骤详情; one CTA per 128-wide latent slice = one MLRA-4
-// branch, groups of 4 CTAs over contiguous tile ranges), but the cache tile is never
-// rewritten: the absorbed query is carried as two bf16 terms q~ = q_hi + q_lo
-// (q_lo = bf16(q~ - q_hi), together ~16 significant bits), and every score is the fp32
-// sum of two bf16 MMAs against the same bf16 tile.  P is rounded to bf16 for P.V.
+// branch, groups of 4 CTAs over contiguous tile ranges), but the latent part of the
+// cache tile is never rewritten: the absorbed query is carried as two bf16 terms
+// q~ = q_hi + q_lo (q_lo = bf16(q~ - q_hi), together ~16 significant bits), and every
+// latent score is the fp32 sum of two bf16 MMAs against the same bf16 tile.  The rope
+// part is scored once in fp16: a converter warp rewrites the tile's 64-column rope box
+// as fp16 in place and the rope query is fp16.  P is rounded to bf16 for P.V.
 //
 // TMEM (512 columns, NT = 128): O [0,128) | S [128,256) | P (bf16 pairs) [256,320) |
-//                               q_hi [320,416) | q_lo [416,512).
+//                               q_hi [320,384) | q_lo [384,448) | q_rope fp16 [448,480).
 // S and P are separate buffers: the QK of tile j+1 may start as soon as the softmax has
 // copied S(j) into registers, and P(j+1) is written once P.V of tile j has completed.
 //
-// Warp roles (11 warps):
+// Warp roles (12 warps):
 //   0-3  softmax half 0 (thread = head row = TMEM lane): score columns [0, NT/2), O [0, 64)
 //   4-7  softmax half 1: score columns [NT/2, NT), O [64, 128); the halves agree on each
 //        row's tile max through shared memory
 //   8    TMA producer
 //   9    TMEM allocator + QK issuer
 //   10   P.V issuer
+//   11   rope-box converter (bf16 -> fp16)
 // The two MMA streams touch disjoint TMEM (S vs P and O), so a burst of QK instructions
 // waiting for the tensor pipe never delays the P.V that a finished softmax released.
 #include <cstdint>
@@ -50,15 +53,16 @@ struct SplitCfg {
   static constexpr int TMEM_O = 0;
   static constexpr int TMEM_S = 128;
   static constexpr int TMEM_P = TMEM_S + NT;
-  static constexpr int TMEM_QH = TMEM_P + NT / 2;
-  static constexpr int TMEM_QL = TMEM_QH + QK_DIMS / 2;
+  static constexpr int TMEM_QH = TMEM_P + NT / 2;  // latent query, bf16 hi term (W/2 columns)
+  static constexpr int TMEM_QL = TMEM_QH + W / 2;  // latent query, bf16 lo term
+  static constexpr int TMEM_QR = TMEM_QL + W / 2;  // rope query, fp16 (32 columns)
   static constexpr int TMEM_COLS = 512;
-  static constexpr int THREADS = 352;
+  static constexpr int THREADS = 384;
   static constexpr int BAR_BYTES = 512;
   static constexpr int RED_BYTES = (2 * 2 * 128 + 2 * 128) * 4;
   static constexpr int MISC_BYTES = BAR_BYTES + RED_BYTES + 4 * (kMaxBatch + 1);
   static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + MISC_BYTES;
-  static_assert(TMEM_QL + QK_DIMS / 2 <= TMEM_COLS, "TMEM budget");
+  static_assert(TMEM_QR + 32 <= TMEM_COLS, "TMEM budget");
   static_assert(NT % 32 == 0 && NT <= 128, "tile rows");
   static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 };
@@ -102,7 +106,7 @@ struct TileCursor {
 };
 
 template <int NT_, int STAGES_>
-__global__ void __launch_bounds__(352, 1)
+__global__ void __launch_bounds__(384, 1)
 decode_split_kernel(const __grid_constant__ CUtensorMap map_ckv, const __grid_constant__ CUtensorMap map_krope,
                     const DecodeArgs a) {
   using C = SplitCfg<NT_, STAGES_>;
@@ -120,7 +124,8 @@ decode_split_kernel(const __grid_constant__ CUtensorMap map_ckv, const __grid_co
   uint64_t* red_bar = q_ready + 1;   // [2] row-max exchange between the softmax halves
   uint64_t* lsum_bar = red_bar + 2;  // row-sum exchange, once per segment
   uint64_t* drain = lsum_bar + 1;    // [2] one per MMA issuer
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 2);
+  uint64_t* conv = drain + 2;        // [STAGES] the stage's rope box is fp16
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(conv + STAGES);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   float* red_max = reinterpret_cast<float*>(misc + C::BAR_BYTES);  // [2 buf][2 half][128]
   float* red_l = red_max + 2 * 2 * 128;                              // [2 half][128]
@@ -141,6 +146,7 @@ decode_split_kernel(const __grid_constant__ CUtensorMap map_ckv, const __grid_co
     for (int i = 0; i < STAGES; ++i) {
       mbar_init(&full[i], 1);
       mbar_init(&empty[i], 1);
+      mbar_init(&conv[i], 1);
     }
     mbar_init(s_full, 1);
     mbar_init(s_free, 8);
@@ -233,6 +239,7 @@ decode_split_kernel(const __grid_constant__ CUtensorMap map_ckv, const __grid_co
     // ------------------------------------------------------------------ QK issuer
     if (lane == 0) {
       constexpr uint32_t idesc_qk = idesc_bf16_f32(128, NT, false);
+      constexpr uint32_t idesc_rope = idesc_f16_f32(128, NT, false);
       const uint32_t tiles_addr = smem_u32(tiles);
       TileCursor qc;
       qc.init(prefix, B, t_begin, t_end, s_first);
@@ -250,10 +257,21 @@ decode_split_kernel(const __grid_constant__ CUtensorMap map_ckv, const __grid_co
         const uint32_t k_base = tiles_addr + (qi % STAGES) * C::STAGE_BYTES;
         const uint32_t d_tmem = tmem + C::TMEM_S;
 #pragma unroll
-        for (int k = 0; k < C::QK_DIMS / 16; ++k) {
+        for (int k = 0; k < C::W / 16; ++k) {  // latent part: bf16 cache x two bf16 query terms
           const uint64_t bdesc = smem_desc_sw128(k_base + (k >> 2) * C::BOX_BYTES + (k & 3) * 32, 16, 1024);
           umma_f16_ts(d_tmem, tmem + C::TMEM_QH + k * 8, bdesc, idesc_qk, k > 0 ? 1u : 0u);
           umma_f16_ts(d_tmem, tmem + C::TMEM_QL + k * 8, bdesc, idesc_qk, 1u);
+        }
+        // rope part: the converter warp has rewritten the stage's rope box as fp16
+        if (!mbar_wait(&conv[qi % STAGES], (qi / STAGES) & 1, limit, abort_flag, status, 16)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const uint64_t bdesc = smem_desc_sw128(k_base + 2 * C::BOX_BYTES + k * 32, 16, 1024);
+          umma_f16_ts(d_tmem, tmem + C::TMEM_QR + k * 8, bdesc, idesc_rope, 1u);
         }
         umma_commit(s_full);
       }
@@ -296,6 +314,27 @@ decode_split_kernel(const __grid_constant__ CUtensorMap map_ckv, const __grid_co
         mbar_wait(&drain[1], 0, limit, &never, status, 15);
       }
     }
+  } else if (warp == 11) {
+    // ------------------------------------------------------------------ rope converter
+    // Rewrites each stage's rope box (bf16 K_R, 128 rows x 64) as fp16 in place, for the
+    // fp16 rope MMAs.  The conversion is exact for |values| < 65504.
+    const int ntiles = t_end - t_begin;
+    for (int it = 0; it < ntiles; ++it) {
+      const int stage = it % STAGES;
+      if (!warp_wait(&full[stage], (it / STAGES) & 1, limit, abort_flag, status, 20)) break;
+      uint4* r = reinterpret_cast<uint4*>(tiles + stage * C::STAGE_BYTES + 2 * C::BOX_BYTES);
+#pragma unroll 4
+      for (int e = lane; e < C::BOX_BYTES / 16; e += 32) {
+        uint4 v = r[e];
+        v.x = bf16x2_to_f16x2(v.x);
+        v.y = bf16x2_to_f16x2(v.y);
+        v.z = bf16x2_to_f16x2(v.z);
+        v.w = bf16x2_to_f16x2(v.w);
+        r[e] = v;
+      }
+      fence_proxy_async_smem();
+      warp_arrive(&conv[stage]);
+    }
   } else if (warp < 8) {
     // ------------------------------------------------------------------ softmax + epilogue
     // The absorbed query comes from the previous kernel, and the split partials written
@@ -323,15 +362,15 @@ decode_split_kernel(const __grid_constant__ CUtensorMap map_ckv, const __grid_co
         const uint4* src = reinterpret_cast<const uint4*>((half == 0 ? q_hi : q_lo) + base);
         const uint32_t col = half == 0 ? C::TMEM_QH : C::TMEM_QL;
 #pragma unroll 1
-        for (int c = 0; c < 3; ++c) {
-          const int e0 = c < 2 ? slice * 128 + 64 * c : 512;  // bf16 element
+        for (int c = 0; c < 2 + (half == 0); ++c) {  // latent chunks, then (half 0) the fp16 rope
+          const int e0 = c < 2 ? slice * 128 + 64 * c : 512;  // 16-bit element
           uint32_t w[32];
 #pragma unroll
           for (int u = 0; u < 8; ++u) {
             const uint4 v = live ? __ldg(src + (e0 >> 3) + u) : make_uint4(0u, 0u, 0u, 0u);
             w[4 * u + 0] = v.x; w[4 * u + 1] = v.y; w[4 * u + 2] = v.z; w[4 * u + 3] = v.w;
           }
-          tmem_st32(t_row + col + 32 * c, w);
+          tmem_st32(t_row + (c < 2 ? col + 32 * c : C::TMEM_QR), w);
         }
         tmem_st_wait();
         tc_fence_before();

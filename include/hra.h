@@ -23,8 +23,9 @@
  * Bounded device waits that expire write a status word in the workspace, read back
  * by hra_check_device_status().
  * Numerics: bf16 inputs, fp32 accumulation; softmax, combine and up-projection in fp32.
- * n_branch = 4: the tensor cores read the bf16 cache as stored, against the absorbed
- * query carried as two bf16 terms (hi + lo, ~16 significant bits).
+ * n_branch = 4: the tensor cores read the latent part of the cache as stored, against
+ * the absorbed query carried as two bf16 terms (hi + lo, ~16 significant bits); the rope
+ * part (query and K_RoPE tile) is scored in fp16, so |K_RoPE values| must stay below 65504.
  * n_branch = 1, 2: the cache tile is converted to fp16 in shared memory and the query is
  * fp16, so |cache values| must stay below 65504.
  * Stream order: the kernels of a call are chained with programmatic dependent launch, so
