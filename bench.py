@@ -112,7 +112,11 @@ class ClockSampler:
                 try:
                     clk = pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM)
                     rs = pynvml.nvmlDeviceGetCurrentClocksEventReasons(h)
-                    self.samples.append((clk, rs))
+                    try:
+                        mw = pynvml.nvmlDeviceGetPowerUsage(h)
+                    except Exception:
+                        mw = None
+                    self.samples.append((clk, rs, mw))
                 except Exception:
                     pass
                 self._stop.wait(0.002)
@@ -129,10 +133,12 @@ class ClockSampler:
     def summary(self):
         if not self.samples:
             return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": ["unsampled"]}
-        clks = sorted(c for c, _ in self.samples)
-        reasons = sorted({n for _, r in self.samples for n, bit in self.REASONS.items() if r & bit})
+        clks = sorted(c for c, _, _ in self.samples)
+        reasons = sorted({n for _, r, _ in self.samples for n, bit in self.REASONS.items() if r & bit})
+        watts = [w / 1000.0 for _, _, w in self.samples if w is not None]
         return {"sm_mhz": statistics.median(clks), "sm_max_mhz": self.max_mhz, "sm_mhz_min": clks[0],
-                "reasons": reasons, "samples": len(clks), "source": "NVML, 2 ms period, timed region only"}
+                "reasons": reasons, "power_w": statistics.median(watts) if watts else None,
+                "samples": len(clks), "source": "NVML, 2 ms period, timed region only"}
 
 
 def time_oracle_sample(wl: synth.Workload, n_seqs: int, n_heads: int):
