@@ -1,8 +1,8 @@
 #!/usr/bin/env python
 """Decode-step benchmark: single-token MLRA-4 decode over a latent KV cache on B200.
 
-A step is one whole decode call (absorb_q -> split-KV decode -> combine/up-projection)
-over one batch of the workload; inputs are resident in HBM when the timed region
+A step is one whole decode call (query absorption -> split-KV decode -> log-sum-exp merge
+-> up-projection, four kernels) over one batch of the workload; inputs are resident in HBM when the timed region
 starts.  Default workload: MLRA-4, B=64, h=128, T=32768, 64-token pages with a random
 page table (2.4 GB of KV cache read per step, larger than L2, so no flush is needed).
 
@@ -177,6 +177,21 @@ def workload_config(wl: synth.Workload, lens) -> dict:
             "l2": "inputs larger than L2 (KV cache per step >> 126 MB); no flush"}
 
 
+def max_over_ranks(values, world: int, device) -> list:
+    """Element-wise maximum of `values` over all ranks: the job's time is its slowest
+    rank's.  Needs an initialised default process group when world > 1."""
+    if world == 1:
+        return [float(v) for v in values]
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return [float(x) for x in t.cpu()]
+
+
+def job_tbs(bytes_per_rank: int, world: int, ms_per_step: float) -> float:
+    """Whole-job throughput in TB/s: every rank reads bytes_per_rank per step."""
+    return world * bytes_per_rank / (ms_per_step * 1e-3) / 1e12
+
+
 def dist_setup():
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -333,10 +348,7 @@ def run_native(args, wl, world, rank, local):
     hra.check_device_status(p, stream)
 
     step_ms = elapsed_ms / args.steps
-    if world > 1:
-        t = torch.tensor([step_ms, e2e_ms, decode_ms], device="cuda", dtype=torch.float64)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        step_ms, e2e_ms, decode_ms = (float(x) for x in t.cpu())
+    step_ms, e2e_ms, decode_ms = max_over_ranks([step_ms, e2e_ms, decode_ms], world, "cuda")
     clocks = clk.summary()
 
     if rank == 0:
@@ -347,7 +359,7 @@ def run_native(args, wl, world, rank, local):
         traffic = ncu_traffic(wl.name)
         line = {
             "metric": METRIC,
-            "value": world * kv / (step_ms * 1e-3) / 1e12, "unit": "TB/s",
+            "value": job_tbs(kv, world, step_ms), "unit": "TB/s",
             "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": step_ms, "us_per_step": step_ms * 1e3,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
@@ -374,7 +386,7 @@ def run_native(args, wl, world, rank, local):
                                 "frac": achieved_tflops / pk["bf16_tflops"],
                                 "note": "algorithmic FLOPs (rope scored once, one query term) over the bf16 dense peak"},
             "clocks": clocks,
-            "e2e": {"value": world * kv / (e2e_ms * 1e-3) / 1e12, "unit": "TB/s", "ms_per_step": e2e_ms,
+            "e2e": {"value": job_tbs(kv, world, e2e_ms), "unit": "TB/s", "ms_per_step": e2e_ms,
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": e2e_steps},
             "gpu_launches": 4 * args.steps,  # absorb, decode, merge, up-projection per step
         }

@@ -1,0 +1,80 @@
+"""The N > 1 host path of bench.py on CPU: two gloo ranks (one process each, rendezvous
+on 127.0.0.1).  Every rank decodes its own replica, so the only cross-rank steps are the
+maximum of the per-rank times and the whole-job throughput; both are checked here."""
+import datetime
+import io
+import os
+import socket
+import sys
+import contextlib
+
+import pytest
+import torch
+import torch.multiprocessing as mp
+
+sys.path.insert(0, os.path.dirname(os.path.dirname(os.path.abspath(__file__))))
+
+WORLD = 2
+
+
+def _free_port() -> int:
+    with socket.socket(socket.AF_INET, socket.SOCK_STREAM) as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _rank_main(rank: int, world: int, port: int, queue) -> None:
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank), WORLD_SIZE=str(world),
+                      LOCAL_RANK=str(rank))
+    import bench
+    torch.distributed.init_process_group("gloo", rank=rank, world_size=world,
+                                         timeout=datetime.timedelta(seconds=60))
+    try:
+        setup = bench.dist_setup()
+        # rank r reports times (1 + r, 10 - r, r / 2): the job's are the maxima
+        times = bench.max_over_ranks([1.0 + rank, 10.0 - rank, 0.5 * rank], world, "cpu")
+        tbs = bench.job_tbs(10 ** 12, world, 1000.0)  # 1 TB per rank per 1 s step
+        queue.put((rank, setup, times, tbs))
+        torch.distributed.barrier()
+    finally:
+        torch.distributed.destroy_process_group()
+
+
+def test_two_gloo_ranks_take_the_slowest_time_and_sum_the_bytes():
+    ctx = mp.get_context("spawn")
+    queue = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_rank_main, args=(r, WORLD, port, queue)) for r in range(WORLD)]
+    for p in procs:
+        p.start()
+    try:
+        results = sorted(queue.get(timeout=120) for _ in range(WORLD))
+    finally:
+        for p in procs:
+            p.join(timeout=60)
+            if p.is_alive():
+                p.kill()
+    assert [p.exitcode for p in procs] == [0] * WORLD
+    for rank, setup, times, tbs in results:
+        assert setup == (WORLD, rank, rank)
+        assert times == [float(WORLD), 10.0, 0.5 * (WORLD - 1)]
+        assert tbs == pytest.approx(float(WORLD))
+
+
+def test_single_rank_reduction_is_the_identity():
+    import bench
+    assert bench.max_over_ranks([3, 1.5], 1, "cpu") == [3.0, 1.5]
+    assert bench.job_tbs(6 * 10 ** 9, 1, 1.0) == pytest.approx(6.0)
+
+
+def test_reference_arm_prints_nothing_on_other_ranks():
+    """Under torchrun only rank 0 times the oracle; the other ranks exit without work."""
+    import argparse
+
+    import bench
+    import synth
+    out = io.StringIO()
+    with contextlib.redirect_stdout(out):
+        bench.run_reference(argparse.Namespace(steps=1, warmup=3, ref_seqs=1, ref_heads=1),
+                            synth.WORKLOADS["small_mlra4_h16_t2k"], 2, 1)
+    assert out.getvalue() == ""
