@@ -1,0 +1,40 @@
+"""Plausible mistakes planted in the oracle, in memory, for tests/test_oracle_mutations.py.
+
+Each entry replaces one piece of source text in one oracle function and re-defines that
+function inside oracle.reference (and the oracle package), so that the pins in
+tests/test_oracle_pins.py can be run against a wrong oracle.  Nothing on disk changes.
+"""
+import inspect
+import textwrap
+
+# (function, source text, replacement, the mistake it stands for)
+MUTATIONS = [
+    ("rope_rotate", "x1 * c - x2 * s", "x1 * c + x2 * s", "rotation sign"),
+    ("rope_rotate", "theta ** (-2.0 * j / d)", "theta ** (-1.0 * j / d)", "rotation frequencies"),
+    ("mlra_decode_absorbed", "pos = L - 1", "pos = L", "query position off by one"),
+    ("mlra_decode_absorbed", "alpha_q * alpha_kv * np.einsum", "alpha_q * np.einsum", "alpha_kv dropped from the key"),
+    ("mlra_decode_absorbed", "math.sqrt(d_nope + d_rope) if", "math.sqrt(d_nope) if", "softmax scale"),
+    ("mlra_decode_absorbed", "@ C[:, cols].T + s_rope)", "@ C[:, cols].T)", "rope score dropped"),
+    ("mlra_decode_absorbed", "out += alpha_kv * np.einsum", "out += np.einsum", "alpha_kv dropped from the value"),
+    ("mlra_decode_absorbed", "w_uk[heads], q[heads, :d_nope]", "w_uv[heads], q[heads, :d_nope]", "W_UV used for W_UK"),
+    ("mlra_decode_absorbed", "+= p[b, :, t0:t1] @ C[:, cols]", "+= p[0, :, t0:t1] @ C[:, cols]",
+     "branch 0's weights for every branch"),
+    ("mlra_decode_absorbed", "return sigma * out", "return out", "branch-sum scale dropped"),
+    ("mlra_decode_expanded", "q_n = alpha_q * q[i, :d_nope]", "q_n = q[i, :d_nope]", "alpha_q dropped"),
+    ("mlra_decode_expanded", "K = np.concatenate([K_nope, k_rope], axis=1)",
+     "K = np.concatenate([K_nope, 0 * k_rope], axis=1)", "rope key dropped"),
+    ("mla_decode", "1.0 / math.sqrt(d_qk) if", "1.0 / math.sqrt(d_nope) if", "MLA softmax scale"),
+]
+
+
+def apply(index: int) -> None:
+    """Plant mutation `index` into the imported oracle."""
+    import oracle
+    from oracle import reference
+    name, old, new, _ = MUTATIONS[index]
+    src = textwrap.dedent(inspect.getsource(getattr(reference, name)))
+    if src.count(old) != 1:
+        raise RuntimeError(f"mutation {index}: {old!r} occurs {src.count(old)} times in {name}")
+    exec(compile(src.replace(old, new), f"<mutated {name}>", "exec"), reference.__dict__)
+    if hasattr(oracle, name):
+        setattr(oracle, name, reference.__dict__[name])
