@@ -377,7 +377,7 @@ def run_native(args, wl, world, rank, local):
                                      "each step timed on its own"})),
             "kv_frac_of_nominal_8TBs": kv / (step_ms * 1e-3) / 1e9 / NOMINAL_HBM_GBS,
             "stage_us": {"absorb_q": float(stage_ms[:, 0].mean()) * 1e3, "decode": decode_ms * 1e3,
-                         "combine_upproj": float(stage_ms[:, 2].mean()) * 1e3},
+                         "combine_upproj": float(stage_ms[:, 2].mean()) * 1e3},  # merge + up-projection
             "roofline": {"kernel": "decode_split_kernel" if wl.n_branch == 4 else "decode_kernel", "bound": "hbm", "achieved": achieved_gbs,
                          "peak": pk["hbm_gbs"], "unit": "GB/s", "frac": achieved_gbs / pk["hbm_gbs"],
                          "peak_source": pk_src, "traffic": traffic,

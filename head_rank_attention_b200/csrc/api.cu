@@ -1,6 +1,6 @@
 // api.cu -- the C ABI of libhra.so (declared in include/hra.h): argument validation,
 // workspace layout, TMA descriptor encoding and the launch sequence
-//   absorb_q  ->  decode (split-KV, tcgen05)  ->  combine_upproj
+//   absorb (tcgen05) -> split-KV decode (tcgen05) -> log-sum-exp merge -> up-projection (tcgen05)
 // of one decode step, all on the caller's stream.  Nothing here allocates device memory.
 #include <cuda.h>
 #include <cudaTypedefs.h>

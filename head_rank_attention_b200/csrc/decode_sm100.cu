@@ -3,7 +3,8 @@
 // Step 2 of the decode in "Multi-Head Low-Rank Attention" (方法步骤详情): MQA-style
 // attention of the absorbed per-head queries over the shared key [C_KV | K_RoPE] and
 // value C_KV, one independent softmax per (head, branch) (核心方法:
-// O = sum_b Softmax(Q K_b^T) V_b; MLA is the single-branch case).
+// O = sum_b Softmax(Q K_b^T) V_b; MLA is the single-branch case).  This kernel serves MLA
+// (NB = 1) and MLRA-2 (NB = 2); MLRA-4 runs decode_split_sm100.cu.
 //
 // Work decomposition (one CTA per SM):
 //   blockIdx.x = slice c in 0..3: the CTA owns output latent columns [128c, 128c+128),

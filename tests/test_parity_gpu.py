@@ -69,6 +69,24 @@ def test_many_sequences():
     assert_parity(out.cpu().numpy(), oracle.decode_batch(inp, wl, form="absorbed"), "many")
 
 
+@pytest.mark.parametrize("n_branch", [4, 2, 1])
+def test_maximum_batch(n_branch):
+    """B = 1024 (the largest batch the library takes), mixed lengths including zeros,
+    8 heads: every sequence-indexed table at its largest, absorb and up-projection over
+    8 chunks of 128 sequences."""
+    rng = np.random.default_rng(11)
+    lens = rng.integers(0, 300, size=1024)
+    lens[rng.integers(0, 1024, size=20)] = 0
+    wl = _case(f"maxbatch_{n_branch}", n_branch, tuple(int(x) for x in lens), heads=8)
+    inp = synth.make_inputs(wl)
+    out, _, _ = run_gpu(synth.to_device(inp), wl)
+    got = out.cpu().numpy()
+    zero = lens == 0
+    assert np.all(got[zero] == 0)
+    ref = oracle.decode_batch(inp, wl, seqs=[int(s) for s in np.flatnonzero(~zero)], form="absorbed")
+    assert_parity(got[~zero], ref, wl.name)
+
+
 def test_bf16_output():
     wl = _case("bf16out", 4, (700, 33))
     inp = synth.make_inputs(wl)
