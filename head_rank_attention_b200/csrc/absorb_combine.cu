@@ -1,11 +1,11 @@
 // absorb_combine.cu -- the steps around the split-KV decode, on the tensor cores.
 //
 // absorb ("Multi-Head Low-Rank Attention", 方法步骤详情, step 1 -- query-side weight
-// absorption), one CTA per (head i, chunk of 128 sequences):
+// absorption), one CTA per (head i, chunk of 128 sequences, half of the latent):
 //     q~[s,i,0:512] = alpha_q * alpha_kv * q_nope[s,i] . W_UK[i]^T        (W_UK[i]: 512 x 128)
-// as one tcgen05 pass with M = the chunk's sequences, N = 512 latent (two N = 256
-// halves), K = 128: A = the q_nope rows, B = W_UK[i] (its rows are latent indices, each
-// with 128 contiguous nope dims: K-major), D in all 512 TMEM columns.  bf16 x bf16
+// as one tcgen05 pass with M = the chunk's sequences, N = 256 latent (the CTA's half),
+// K = 128: A = the q_nope rows, B = W_UK[i] (its rows are latent indices, each with 128
+// contiguous nope dims: K-major), D in 256 TMEM columns.  bf16 x bf16
 // products are exact in the fp32 accumulator, so this equals the fp32 definition up to
 // summation order.  A thread of the epilogue owns one sequence and 32 consecutive latent
 // columns at a time, so q~ (fp16, or the two-term bf16 split the MLRA-4 kernel uses) is
@@ -42,9 +42,9 @@ constexpr uint64_t kWaitNs = 1000000000ull;  // 1 s bound on each wait
 // ---------------------------------------------------------------------------- absorb
 struct AbsorbCfg {
   static constexpr int Q_BYTES = 2 * 128 * 128;  // 2 K boxes of [128 sequences x 128 B]
-  static constexpr int W_BYTES = 4 * 256 * 128;  // 2 latent halves x 2 K boxes of [256 rows x 128 B]
+  static constexpr int W_BYTES = 2 * 256 * 128;  // this CTA's latent half: 2 K boxes of [256 rows x 128 B]
   static constexpr int SMEM = 1024 + Q_BYTES + W_BYTES + 32 * 8 + 64;
-  static constexpr int TMEM_COLS = 512;
+  static constexpr int TMEM_COLS = 256;
   static constexpr int THREADS = 256;
 };
 
@@ -74,8 +74,8 @@ __device__ __forceinline__ void store_q32(const AbsorbArgs& a, long long dst, lo
   }
 }
 
-// grid (h, ceil(B / 128)), 256 threads.  Warp w owns the sequences of TMEM lane quadrant
-// w % 4 and latent half w / 4.
+// grid (h, ceil(B / 128), 2 latent halves), 256 threads, two CTAs per SM.  Warp w owns the
+// sequences of TMEM lane quadrant w % 4 and 128 of the CTA's 256 latent columns (w / 4).
 __global__ void __launch_bounds__(AbsorbCfg::THREADS, 1)
 absorb_tc_kernel(const __grid_constant__ CUtensorMap map_wuk, const __grid_constant__ CUtensorMap map_q,
                  const AbsorbArgs a) {
@@ -89,6 +89,7 @@ absorb_tc_kernel(const __grid_constant__ CUtensorMap map_wuk, const __grid_const
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   const int i = blockIdx.x;
   const int s0 = blockIdx.y * 128;
+  const int nh = blockIdx.z;  // latent half [256 nh, +256)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
   if (threadIdx.x == 0) {
@@ -118,20 +119,17 @@ absorb_tc_kernel(const __grid_constant__ CUtensorMap map_wuk, const __grid_const
       mbar_arrive_expect_tx(&bars[0], C::Q_BYTES + C::W_BYTES);
       for (int kb = 0; kb < 2; ++kb)
         tma_load_2d(qbuf + kb * 16384, &map_q, &bars[0], i * 192 + 64 * kb, s0, stream_once);
-      for (int n = 0; n < 2; ++n)
-        for (int kb = 0; kb < 2; ++kb)
-          tma_load_2d(wbuf + (n * 2 + kb) * 32768, &map_wuk, &bars[0], 64 * kb, i * 512 + 256 * n, stream_once);
+      for (int kb = 0; kb < 2; ++kb)
+        tma_load_2d(wbuf + kb * 32768, &map_wuk, &bars[0], 64 * kb, i * 512 + 256 * nh, stream_once);
       if (mbar_wait(&bars[0], 0, kWaitNs, abort_flag, a.status, 40)) {
         tc_fence_after();
         constexpr uint32_t idesc = idesc_bf16_f32(128, 256, false);
         const uint32_t qa = smem_u32(qbuf), wa = smem_u32(wbuf);
-        for (int n = 0; n < 2; ++n) {
 #pragma unroll
-          for (int ks = 0; ks < 8; ++ks) {
-            const uint64_t adesc = smem_desc_sw128(qa + (ks >> 2) * 16384 + (ks & 3) * 32, 16, 1024);
-            const uint64_t bdesc = smem_desc_sw128(wa + (n * 2 + (ks >> 2)) * 32768 + (ks & 3) * 32, 16, 1024);
-            umma_f16_ss(tmem + 256 * n, adesc, bdesc, idesc, ks > 0 ? 1u : 0u);
-          }
+        for (int ks = 0; ks < 8; ++ks) {
+          const uint64_t adesc = smem_desc_sw128(qa + (ks >> 2) * 16384 + (ks & 3) * 32, 16, 1024);
+          const uint64_t bdesc = smem_desc_sw128(wa + (ks >> 2) * 32768 + (ks & 3) * 32, 16, 1024);
+          umma_f16_ss(tmem, adesc, bdesc, idesc, ks > 0 ? 1u : 0u);
         }
       }
       umma_commit(&bars[1]);  // arrives once every MMA issued above (possibly none) completed
@@ -141,16 +139,16 @@ absorb_tc_kernel(const __grid_constant__ CUtensorMap map_wuk, const __grid_const
   // Everything above reads only inputs of the call; what follows writes the workspace,
   // which the previous call's kernels read, so it waits for them.
   grid_dep_wait();
-  if (blockIdx.x == 0 && blockIdx.y == 0) {
+  if (blockIdx.x == 0 && blockIdx.y == 0 && blockIdx.z == 0) {
     if (threadIdx.x < 4) a.status[threadIdx.x] = 0;  // fresh per call
     if (warp == 3) tile_prefix_warp(a.seq_lens, a.batch, a.tile_tokens, a.tile_prefix);
   }
   const int r = 32 * (warp & 3) + lane;  // sequence within the chunk = TMEM lane
   const int s = s0 + r;
-  const int part = warp >> 2;            // latent half [256 part, +256); rope pairs [16 part, +16)
+  const int part = warp >> 2;            // columns [256 nh + 128 part, +128); rope pairs [16 part, +16)
   const long long lo_off = static_cast<long long>(a.batch) * a.heads * 576;
   const long long row = (static_cast<long long>(s) * a.heads + i) * 576;
-  if (s < a.batch) {
+  if (s < a.batch && nh == 0) {
     // RoPE of the query's rope part at position L-1, while the loads and MMAs run: pair
     // (j, j + 32) turns by pos * theta^(-2j/64) radians.  The angle is carried in turns
     // (fp64: pos reaches 2^21); its fractional part is exact and is then evaluated in
@@ -196,10 +194,11 @@ absorb_tc_kernel(const __grid_constant__ CUtensorMap map_wuk, const __grid_const
     const float scale = a.alpha_q * a.alpha_kv;
     const uint32_t lane_base = static_cast<uint32_t>(32 * (warp & 3)) << 16;
 #pragma unroll 1
-    for (int c = 0; c < 8; ++c) {
-      const int k0 = 256 * part + 32 * c;
+    for (int c = 0; c < 4; ++c) {
+      const int col = 128 * part + 32 * c;  // TMEM column = latent column - 256 nh
+      const int k0 = 256 * nh + col;
       uint32_t v[32];
-      tmem_ld32(tmem + lane_base + k0, v);
+      tmem_ld32(tmem + lane_base + col, v);
       tmem_ld_wait();
       if (s < a.batch) {
         float x[32];
@@ -507,7 +506,7 @@ cudaError_t launch_absorb_q(const CUtensorMap& map_wuk, const CUtensorMap& map_q
                             cudaStream_t stream, bool pdl) {
   cudaError_t e = set_smem(absorb_tc_kernel, AbsorbCfg::SMEM);
   if (e != cudaSuccess) return e;
-  return launch_kernel(absorb_tc_kernel, dim3(a.heads, (a.batch + 127) / 128), dim3(AbsorbCfg::THREADS),
+  return launch_kernel(absorb_tc_kernel, dim3(a.heads, (a.batch + 127) / 128, 2), dim3(AbsorbCfg::THREADS),
                        AbsorbCfg::SMEM, stream, pdl, map_wuk, map_q, a);
 }
 
