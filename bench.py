@@ -266,6 +266,7 @@ def run_native(args, wl, world, rank, local):
     # Inputs smaller than twice the L2 (126 MB) would stay cached between steps: flush it
     # by writing a 512 MB buffer before every timed step.
     step_bytes = kv + sum(t.numel() * t.element_size() for t in (dev.q, dev.w_uk, dev.w_uv))
+    step_bytes_all = step_bytes + out.numel() * 4
     flush = torch.zeros(128 << 20, dtype=torch.float32, device="cuda") if step_bytes < (252 << 20) else None
 
     # The timed steps: the call as a user makes it (kernels chained by programmatic
@@ -306,6 +307,15 @@ def run_native(args, wl, world, rank, local):
                 e1.record(stream)
             torch.cuda.synchronize()
             elapsed_ms = sum(e0.elapsed_time(e1) for e0, e1 in pairs)
+    hot_ms = None
+    if flush is not None:  # the same steps back to back with a warm L2, reported beside
+        h0, h1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        h0.record(stream)
+        for k in range(args.steps):
+            one_step()
+        h1.record(stream)
+        torch.cuda.synchronize()
+        hot_ms = h0.elapsed_time(h1) / args.steps
     hra.check_device_status(p, stream)
     del graph
 
@@ -376,6 +386,9 @@ def run_native(args, wl, world, rank, local):
                               {"l2": "inputs smaller than L2: 512 MB written before every step, "
                                      "each step timed on its own"})),
             "kv_frac_of_nominal_8TBs": kv / (step_ms * 1e-3) / 1e9 / NOMINAL_HBM_GBS,
+            # every byte a step must move (KV, both weight tensors, q, out) over the measured copy peak
+            "step_bytes_frac": step_bytes_all / (step_ms * 1e-3) / 1e9 / peaks()[0]["hbm_gbs"],
+            **({} if hot_ms is None else {"us_per_step_hot_l2": hot_ms * 1e3}),
             "stage_us": {"absorb_q": float(stage_ms[:, 0].mean()) * 1e3, "decode": decode_ms * 1e3,
                          "combine_upproj": float(stage_ms[:, 2].mean()) * 1e3},  # merge + up-projection
             "roofline": {"kernel": "decode_split_kernel" if wl.n_branch == 4 else "decode_kernel", "bound": "hbm", "achieved": achieved_gbs,

@@ -115,12 +115,12 @@ absorb_tc_kernel(const __grid_constant__ CUtensorMap map_wuk, const __grid_const
     // warp 0 issues the loads and the MMAs from lane 0; its other lanes wait at the
     // __syncwarp so that no lane of this warp polls a barrier lane 0 has yet to release
     if (lane == 0) {
-      const uint64_t stream_once = l2_policy_evict_first();
+      const uint64_t stream_once = l2_policy_evict_first(), keep = l2_policy_evict_last();
       mbar_arrive_expect_tx(&bars[0], C::Q_BYTES + C::W_BYTES);
       for (int kb = 0; kb < 2; ++kb)
         tma_load_2d(qbuf + kb * 16384, &map_q, &bars[0], i * 192 + 64 * kb, s0, stream_once);
       for (int kb = 0; kb < 2; ++kb)
-        tma_load_2d(wbuf + kb * 32768, &map_wuk, &bars[0], 64 * kb, i * 512 + 256 * nh, stream_once);
+        tma_load_2d(wbuf + kb * 32768, &map_wuk, &bars[0], 64 * kb, i * 512 + 256 * nh, keep);
       if (mbar_wait(&bars[0], 0, kWaitNs, abort_flag, a.status, 40)) {
         tc_fence_after();
         constexpr uint32_t idesc = idesc_bf16_f32(128, 256, false);
@@ -375,7 +375,7 @@ upproj_tc_kernel(const __grid_constant__ CUtensorMap map_wuv, const __grid_const
     // lane 0 streams the four K chunks through two stages and issues the MMAs; the other
     // lanes wait at the __syncwarp
     if (lane == 0) {
-      const uint64_t stream_once = l2_policy_evict_first();
+      const uint64_t stream_once = l2_policy_evict_first(), keep = l2_policy_evict_last();
       const int row_hi = i * a.batch + s0;             // this head's o_lat rows
       const int row_lo = row_hi + a.heads * a.batch;   // the lo term, h*B rows later
       // only the 32-row boxes that hold this chunk's sequences are loaded; the other A
@@ -386,7 +386,7 @@ upproj_tc_kernel(const __grid_constant__ CUtensorMap map_wuv, const __grid_const
         uint64_t* bar = &full[c % C::STAGES];
         mbar_arrive_expect_tx(bar, 4 * nbox * 4096 + C::B_BYTES);
         for (int db = 0; db < 2; ++db)
-          tma_load_2d(st + C::A_BYTES + db * 16384, &map_wuv, bar, 64 * db, i * 512 + 128 * c, stream_once);
+          tma_load_2d(st + C::A_BYTES + db * 16384, &map_wuv, bar, 64 * db, i * 512 + 128 * c, keep);
       };
       auto load_o = [&](int c) {  // o_lat rows of chunk c, written by the merge kernel
         uint8_t* st = stages + (c % C::STAGES) * C::STAGE_BYTES;
