@@ -11,6 +11,11 @@ page table (2.4 GB of KV cache read per step, larger than L2, so no flush is nee
 Multi-GPU (torchrun, one rank per GPU): every rank decodes its own replica batch (the
 path has no exchange step); value = all ranks' KV bytes / max-over-ranks step time.
 One JSON line is printed by rank 0.
+
+--tp W (W = 2 or 4, MLRA-4 workloads): tensor parallelism by branch.  Rank r holds its
+W-th of the branches (cache columns + K_RoPE, W_UK / W_UV rows) and a step is its shard's
+decode followed by an NCCL all-reduce of out; run it with --gpus W.  With one GPU, the
+rank-0 shard's step is timed alone (no all-reduce).
 """
 from __future__ import annotations
 
@@ -43,12 +48,12 @@ DECODE_SOURCES = ["head_rank_attention_b200/csrc/decode_split_sm100.cu", "head_r
                   "head_rank_attention_b200/csrc/decode_sm100.h"]
 
 
-def tensor_flops_per_token(n_branch: int, heads: int) -> int:
-    """Tensor-core FLOPs per cached token the decode kernel issues: each of the 4 slice
-    CTAs scores over its branch (w + 64 dims) for 128 padded head rows, and P.V adds
-    2*512 per head row.  Algorithmic count (shared rope scored once, real heads only):
-    2*(512+64)*h + 2*512*h."""
-    return 2 * (512 + 64) * heads + 2 * 512 * heads
+def tensor_flops_per_token(n_branch: int, heads: int, d_c: int = 512) -> int:
+    """Algorithmic tensor-core FLOPs per cached token (shared rope scored once, real heads
+    only, one query term): scores over d_c + 64 dims and P.V over d_c columns per head,
+    2*(d_c+64)*h + 2*d_c*h.  (The kernels issue more: each slice CTA scores its branch
+    for 128 padded head rows, and MLRA-4 scores with two query terms.)"""
+    return 2 * (d_c + 64) * heads + 2 * d_c * heads
 
 
 def peaks():
@@ -141,10 +146,12 @@ class ClockSampler:
                 "samples": len(clks), "source": "NVML, 2 ms period, timed region only"}
 
 
-def time_oracle_sample(wl: synth.Workload, n_seqs: int, n_heads: int):
+def time_oracle_sample(wl: synth.Workload, n_seqs: int, n_heads: int, tp_world: int = 0):
     """Run the fp64 oracle (the expanded definition) on n_seqs x n_heads outputs of the
-    workload; return (seconds, (seq, head) pairs done, threads used)."""
+    workload (of its rank-0 branch shard under tp_world-way tensor parallelism, if set);
+    return (seconds, the sample's share of the step, threads used, sequences, heads)."""
     import oracle
+    from head_rank_attention_b200 import tp
     try:
         import threadpoolctl
         threads = max(i.get("num_threads", 1) for i in threadpoolctl.threadpool_info())
@@ -156,10 +163,15 @@ def time_oracle_sample(wl: synth.Workload, n_seqs: int, n_heads: int):
     seqs = list(range(min(n_seqs, wl.batch)))
     heads = list(range(min(n_heads, wl.heads)))
     rows = {s: synth.seq_rows(wl, s) for s in seqs}  # generation is not timed
+    d_c, n_branch = synth.D_C, wl.n_branch
+    if tp_world:
+        rows = {s: tp.shard_cache(r, 0, tp_world) for s, r in rows.items()}
+        w_uk, w_uv = tp.shard_weights(w_uk, w_uv, 0, tp_world)
+        d_c, n_branch = synth.D_C // tp_world, wl.n_branch // tp_world
     t0 = time.perf_counter()
     for s in seqs:
         r = rows[s]
-        oracle.mlra_decode_expanded(q[s], r[:, :synth.D_C], r[:, synth.D_C:], w_uk, w_uv, wl.n_branch,
+        oracle.mlra_decode_expanded(q[s], r[:, :d_c], r[:, d_c:], w_uk, w_uv, n_branch,
                                     alpha_q=wl.alpha_q, alpha_kv=wl.alpha_kv, branch_scale=wl.sigma_o,
                                     softmax_scale=wl.softmax_scale, rope_theta=wl.rope_theta, heads=heads)
     dt = time.perf_counter() - t0
@@ -168,12 +180,13 @@ def time_oracle_sample(wl: synth.Workload, n_seqs: int, n_heads: int):
     return dt, frac, threads, len(seqs), len(heads)
 
 
-def workload_config(wl: synth.Workload, lens) -> dict:
+def workload_config(wl: synth.Workload, lens, tp_world: int = 0) -> dict:
     return {"workload": wl.name, "variant": {1: "MLA", 2: "MLRA-2", 4: "MLRA-4"}[wl.n_branch],
             "batch": wl.batch, "heads": wl.heads, "seq_len": wl.seq_len,
             "seq_len_min": wl.seq_len_min, "total_tokens": int(np.asarray(lens, dtype=np.int64).sum()),
             "layout": f"paged({wl.page_size})" if wl.page_size else "contiguous",
-            "d_c": 512, "d_rope": 64, "alpha_q": wl.alpha_q, "alpha_kv": wl.alpha_kv, "branch_scale": wl.sigma_o,
+            "d_c": 512 // tp_world if tp_world else 512, "d_rope": 64,
+            **({"tp_shard": f"{4 // tp_world} of 4 branches per rank"} if tp_world else {}), "alpha_q": wl.alpha_q, "alpha_kv": wl.alpha_kv, "branch_scale": wl.sigma_o,
             "l2": "inputs larger than L2 (KV cache per step >> 126 MB); no flush"}
 
 
@@ -203,13 +216,15 @@ def run_reference(args, wl, world, rank):
     if rank != 0:
         return
     lens = synth.seq_lens(wl)
-    kv = synth.kv_bytes(lens)
+    tpw = getattr(args, "tp", 0)
+    d_c = synth.D_C // tpw if tpw else synth.D_C
+    kv = int(np.asarray(lens, dtype=np.int64).sum()) * (d_c + synth.D_ROPE) * 2
     for _ in range(args.warmup):
-        time_oracle_sample(wl, 1, 1)
+        time_oracle_sample(wl, 1, 1, tpw)
     times = []
     frac = threads = None
     for _ in range(args.steps):
-        dt, frac, threads, ns, nh = time_oracle_sample(wl, args.ref_seqs, args.ref_heads)
+        dt, frac, threads, ns, nh = time_oracle_sample(wl, args.ref_seqs, args.ref_heads, tpw)
         times.append(dt / frac)  # extrapolated seconds per full decode step
     step_s = statistics.mean(times)
     value = kv / step_s / 1e12
@@ -217,8 +232,8 @@ def run_reference(args, wl, world, rank):
               f"head(s) of the workload, extrapolated by cached tokens x heads to the full step")
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "TB/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": step_s * 1e3,
-            "us_per_step": step_s * 1e6, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-            "dtype": "f64", "data": "synthetic", "config": workload_config(wl, lens),
+            "us_per_step": step_s * 1e6, "higher_is_better": True, "scaling": "strong" if tpw else "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic", "config": workload_config(wl, lens, tpw),
             "cpu_baseline": {"value": value, "unit": "TB/s", "cores": threads, "kind": "oracle", "sample": sample},
             "e2e": {"value": value, "unit": "TB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
@@ -235,12 +250,26 @@ def run_native(args, wl, world, rank, local):
 
     inp = synth.make_inputs(wl)
     lens = inp.seq_lens.numpy()
-    kv = synth.kv_bytes(lens)
     dev = synth.to_device(inp)
+    tpw = args.tp
+    all_reduce = tpw > 0 and world > 1
+    d_c, n_branch = synth.D_C, wl.n_branch
+    cache, w_uk, w_uv = dev.cache, dev.w_uk, dev.w_uv
+    host_cache, host_wuk, host_wuv = inp.cache, inp.w_uk, inp.w_uv
+    if tpw:  # this rank's branch shard (rank 0's when one GPU stands alone)
+        shard = rank if world == tpw else 0
+        cache = hra.tp.shard_cache(dev.cache, shard, tpw)
+        w_uk, w_uv = hra.tp.shard_weights(dev.w_uk, dev.w_uv, shard, tpw)
+        host_cache = hra.tp.shard_cache(inp.cache, shard, tpw)
+        host_wuk, host_wuv = hra.tp.shard_weights(inp.w_uk, inp.w_uv, shard, tpw)
+        dev.cache = dev.w_uk = dev.w_uv = None
+        torch.cuda.empty_cache()
+        d_c, n_branch = synth.D_C // tpw, wl.n_branch // tpw
+    kv = int(lens.astype(np.int64).sum()) * (d_c + synth.D_ROPE) * 2  # cache bytes this rank reads
     stream = torch.cuda.current_stream()
     out = torch.empty(wl.batch, wl.heads, synth.D_V, dtype=torch.float32, device="cuda")
-    p = hra.make_params(dev.q, dev.ckv, dev.krope, dev.seq_lens, dev.w_uk, dev.w_uv, out,
-                        n_branch=wl.n_branch, alpha_q=wl.alpha_q, alpha_kv=wl.alpha_kv, branch_scale=wl.sigma_o,
+    p = hra.make_params(dev.q, cache[:, :d_c], cache[:, d_c:], dev.seq_lens, w_uk, w_uv, out,
+                        n_branch=n_branch, alpha_q=wl.alpha_q, alpha_kv=wl.alpha_kv, branch_scale=wl.sigma_o,
                         softmax_scale=wl.softmax_scale, rope_theta=wl.rope_theta, block_table=dev.block_table,
                         page_size=wl.page_size, seq_stride=dev.seq_stride, num_splits=args.num_splits)
     ws = hra.alloc_workspace(p)
@@ -254,8 +283,13 @@ def run_native(args, wl, world, rank, local):
     handles = [(ctypes.c_void_p * 4)(*[e.cuda_event for e in evs]) for evs in events]
     assert all(h for hs in handles for h in hs), "CUDA events were not created"
 
-    for _ in range(args.warmup):
+    def call():  # one step as a user makes it: the decode call (+ the all-reduce under TP)
         hra.mlra_decode(p, stream)
+        if all_reduce:
+            hra.tp.all_reduce_out(out)
+
+    for _ in range(args.warmup):
+        call()
     hra.check_device_status(p, stream)
 
     def barrier():
@@ -265,7 +299,7 @@ def run_native(args, wl, world, rank, local):
 
     # Inputs smaller than twice the L2 (126 MB) would stay cached between steps: flush it
     # by writing a 512 MB buffer before every timed step.
-    step_bytes = kv + sum(t.numel() * t.element_size() for t in (dev.q, dev.w_uk, dev.w_uv))
+    step_bytes = kv + sum(t.numel() * t.element_size() for t in (dev.q, w_uk, w_uv))
     step_bytes_all = step_bytes + out.numel() * 4
     flush = torch.zeros(128 << 20, dtype=torch.float32, device="cuda") if step_bytes < (252 << 20) else None
 
@@ -273,7 +307,7 @@ def run_native(args, wl, world, rank, local):
     # dependent launch), replayed from a CUDA graph of one call unless --no-graph, so that
     # host-side launch work does not bound the short configurations.
     graph = None
-    if not args.no_graph:
+    if not args.no_graph and not all_reduce:
         graph = torch.cuda.CUDAGraph()
         with torch.cuda.graph(graph):
             hra.mlra_decode(p, torch.cuda.current_stream())
@@ -285,7 +319,7 @@ def run_native(args, wl, world, rank, local):
         if graph is not None:
             graph.replay()
         else:
-            hra.mlra_decode(p, stream)
+            call()
 
     barrier()
     with ClockSampler(dev_id) as clk:
@@ -317,6 +351,7 @@ def run_native(args, wl, world, rank, local):
         torch.cuda.synchronize()
         hot_ms = h0.elapsed_time(h1) / args.steps
     hra.check_device_status(p, stream)
+    graph_used = graph is not None
     del graph
 
     # Per-stage breakdown (and the decode kernel's own time for the roofline): the same
@@ -334,12 +369,12 @@ def run_native(args, wl, world, rank, local):
     decode_ms = float(stage_ms[:, 1].mean())
 
     # end to end through the C ABI with host buffers: H2D of every input, decode, D2H of out
-    pin = {k: v.pin_memory() for k, v in dict(q=inp.q, cache=inp.cache, seq_lens=inp.seq_lens,
-                                               w_uk=inp.w_uk, w_uv=inp.w_uv).items()}
+    pin = {k: v.pin_memory() for k, v in dict(q=inp.q, cache=host_cache, seq_lens=inp.seq_lens,
+                                               w_uk=host_wuk, w_uv=host_wuv).items()}
     if inp.block_table is not None:
         pin["block_table"] = inp.block_table.pin_memory()
     host_out = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
-    dmap = dict(q=dev.q, cache=dev.cache, seq_lens=dev.seq_lens, w_uk=dev.w_uk, w_uv=dev.w_uv,
+    dmap = dict(q=dev.q, cache=cache, seq_lens=dev.seq_lens, w_uk=w_uk, w_uv=w_uv,
                 block_table=dev.block_table)
     h2d = sum(t.numel() * t.element_size() for t in pin.values())
     d2h = host_out.numel() * host_out.element_size()
@@ -350,7 +385,7 @@ def run_native(args, wl, world, rank, local):
     for _ in range(e2e_steps):
         for k, t in pin.items():
             dmap[k].copy_(t, non_blocking=True)
-        hra.mlra_decode(p, stream)
+        call()
         host_out.copy_(out, non_blocking=True)
     e1.record(stream)
     torch.cuda.synchronize()
@@ -364,24 +399,29 @@ def run_native(args, wl, world, rank, local):
     if rank == 0:
         pk, pk_src = peaks()
         achieved_gbs = kv / (decode_ms * 1e-3) / 1e9
-        flops = tensor_flops_per_token(wl.n_branch, wl.heads) * int(lens.astype(np.int64).sum())
+        flops = tensor_flops_per_token(n_branch, wl.heads, d_c) * int(lens.astype(np.int64).sum())
         achieved_tflops = flops / (decode_ms * 1e-3) / 1e12
-        traffic = ncu_traffic(wl.name)
+        traffic = ncu_traffic(f"{wl.name}/tp{tpw}" if tpw else wl.name)
+        if tpw:
+            parallelism = (f"tp{tpw}: branch shards + NCCL all-reduce of out" if all_reduce else
+                           f"tp{tpw}: rank 0's branch shard alone (no all-reduce)")
+        else:
+            parallelism = f"replicas x{world}" if world > 1 else "1 GPU"
         line = {
             "metric": METRIC,
             "value": job_tbs(kv, world, step_ms), "unit": "TB/s",
             "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": step_ms, "us_per_step": step_ms * 1e3,
-            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "higher_is_better": True, "scaling": "strong" if tpw else "weak", "vs_baseline": None,
             "dtype": "bf16" if wl.n_branch == 4 else "f16",
             "precision": ("bf16 inputs; bf16 tensor-core operands, the absorbed query as two bf16 terms; "
                           "fp32 accumulate, softmax, combine") if wl.n_branch == 4 else
                          ("bf16 inputs; fp16 tensor-core operands (cache tile converted in shared memory); "
                           "fp32 accumulate, softmax, combine"),
             "data": "synthetic",
-            "config": dict(workload_config(wl, lens), parallelism=f"replicas x{world}" if world > 1 else "1 GPU",
-                           num_splits=args.num_splits or "auto (SMs/4)",
-                           timing="CUDA-graph replays of one call" if not args.no_graph else "direct calls",
+            "config": dict(workload_config(wl, lens, tpw), parallelism=parallelism,
+                           num_splits=args.num_splits or f"auto (SMs/{d_c // 128})",
+                           timing="CUDA-graph replays of one call" if graph_used else "direct calls",
                            **({} if flush is None else
                               {"l2": "inputs smaller than L2: 512 MB written before every step, "
                                      "each step timed on its own"})),
@@ -391,7 +431,8 @@ def run_native(args, wl, world, rank, local):
             **({} if hot_ms is None else {"us_per_step_hot_l2": hot_ms * 1e3}),
             "stage_us": {"absorb_q": float(stage_ms[:, 0].mean()) * 1e3, "decode": decode_ms * 1e3,
                          "combine_upproj": float(stage_ms[:, 2].mean()) * 1e3},  # merge + up-projection
-            "roofline": {"kernel": "decode_split_kernel" if wl.n_branch == 4 else "decode_kernel", "bound": "hbm", "achieved": achieved_gbs,
+            "roofline": {"kernel": "decode_split_kernel" if d_c // n_branch == 128 else "decode_kernel",
+                         "bound": "hbm", "achieved": achieved_gbs,
                          "peak": pk["hbm_gbs"], "unit": "GB/s", "frac": achieved_gbs / pk["hbm_gbs"],
                          "peak_source": pk_src, "traffic": traffic,
                          "bytes_per_launch": kv},
@@ -404,7 +445,7 @@ def run_native(args, wl, world, rank, local):
             "gpu_launches": 4 * args.steps,  # absorb, decode, merge, up-projection per step
         }
         if world == 1 and not args.no_cpu_baseline:
-            dt, frac, threads, ns, nh = time_oracle_sample(wl, args.cpu_seqs, args.cpu_heads)
+            dt, frac, threads, ns, nh = time_oracle_sample(wl, args.cpu_seqs, args.cpu_heads, tpw)
             cpu_step = dt / frac
             line["cpu_baseline"] = {
                 "value": kv / cpu_step / 1e12, "unit": "TB/s", "cores": threads, "kind": "oracle",
@@ -433,11 +474,17 @@ def main():
     ap.add_argument("--ref-heads", type=int, default=8)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-graph", action="store_true", help="time direct calls instead of CUDA-graph replays")
+    ap.add_argument("--tp", type=int, default=0, choices=[0, 2, 4],
+                    help="tensor parallelism by branch over this many ranks (MLRA-4 workloads)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     world, rank, local = dist_setup()
     wl = synth.WORKLOADS[args.workload]
+    if args.tp and wl.n_branch != 4:
+        ap.error("--tp needs an MLRA-4 workload (128-wide branches)")
+    if args.tp and world not in (1, args.tp):
+        ap.error(f"--tp {args.tp} runs on {args.tp} ranks (or one GPU for a single shard), not {world}")
     if args.impl == "reference":
         run_reference(args, wl, world, rank)
     else:

@@ -1,9 +1,11 @@
 // absorb_combine.cu -- the steps around the split-KV decode, on the tensor cores.
 //
 // absorb ("Multi-Head Low-Rank Attention", 方法步骤详情, step 1 -- query-side weight
-// absorption), one CTA per (head i, chunk of 128 sequences, half of the latent):
-//     q~[s,i,0:512] = alpha_q * alpha_kv * q_nope[s,i] . W_UK[i]^T        (W_UK[i]: 512 x 128)
-// as one tcgen05 pass with M = the chunk's sequences, N = 256 latent (the CTA's half),
+// absorption), one CTA per (head i, chunk of 128 sequences, 256 columns of the latent):
+//     q~[s,i,0:d_c] = alpha_q * alpha_kv * q_nope[s,i] . W_UK[i]^T        (W_UK[i]: d_c x 128)
+// with d_c = 512, or 256 / 128 when the call holds a shard of 128-wide branches (tensor
+// parallelism by branch, 核心方法: under 4-way TP each device holds one MLRA-4 branch).
+// One tcgen05 pass with M = the chunk's sequences, N = min(d_c, 256) latent (the CTA's part),
 // K = 128: A = the q_nope rows, B = W_UK[i] (its rows are latent indices, each with 128
 // contiguous nope dims: K-major), D in 256 TMEM columns.  bf16 x bf16
 // products are exact in the fp32 accumulator, so this equals the fp32 definition up to
@@ -11,19 +13,19 @@
 // columns at a time, so q~ (fp16, or the two-term bf16 split the MLRA-4 kernel uses) is
 // written with 16-byte stores.  The same threads rotate q_rope to position L-1.  The
 // branch structure needs no special case: branch b's absorbed query is columns
-// [b*w, (b+1)*w) of the same 512-vector (W_UK^(b),(i) is the matching row block).
+// [b*w, (b+1)*w) of the same d_c-vector (W_UK^(b),(i) is the matching row block).
 //
 // merge (step 2b): the split-KV partial states of a (sequence, 128-wide latent slice,
 // head) are combined by log-sum-exp, o = sum_g 2^(m_g - M) O_g / sum_g 2^(m_g - M) l_g,
 // and o_lat is stored as bf16 hi + lo terms.
 //
 // upproj (step 3), one CTA per (head i, chunk of 128 sequences):
-//     out[s,i,:] = branch_scale * alpha_kv * o_lat[s,i,:] . W_UV[i]        (W_UV[i]: 512 x 128)
-// M = sequences, N = 128 output columns, K = 512 latent (both o_lat terms): A = o_lat
+//     out[s,i,:] = branch_scale * alpha_kv * o_lat[s,i,:] . W_UV[i]        (W_UV[i]: d_c x 128)
+// M = sequences, N = 128 output columns, K = d_c latent (both o_lat terms): A = o_lat
 // rows (K-major), B = W_UV[i] read MN-major (its rows are latent indices with the 128
-// output columns contiguous), streamed through two shared-memory stages in four K
+// output columns contiguous), streamed through two shared-memory stages in d_c / 128 K
 // chunks.  The branches partition the latent, so summing the per-branch up-projections
-// is this one contraction.
+// is this one contraction (and a branch shard's output is its part of that sum).
 #include <cstdint>
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
@@ -74,8 +76,9 @@ __device__ __forceinline__ void store_q32(const AbsorbArgs& a, long long dst, lo
   }
 }
 
-// grid (h, ceil(B / 128), 2 latent halves), 256 threads, two CTAs per SM.  Warp w owns the
-// sequences of TMEM lane quadrant w % 4 and 128 of the CTA's 256 latent columns (w / 4).
+// grid (h, ceil(B / 128), max(d_c / 256, 1) latent parts), 256 threads, two CTAs per SM.
+// Warp w owns the sequences of TMEM lane quadrant w % 4 and 128 of the CTA's
+// min(d_c, 256) latent columns (w / 4; with 128 columns warps 4-7 only rotate q_rope).
 __global__ void __launch_bounds__(AbsorbCfg::THREADS, 1)
 absorb_tc_kernel(const __grid_constant__ CUtensorMap map_wuk, const __grid_constant__ CUtensorMap map_q,
                  const AbsorbArgs a) {
@@ -89,7 +92,9 @@ absorb_tc_kernel(const __grid_constant__ CUtensorMap map_wuk, const __grid_const
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   const int i = blockIdx.x;
   const int s0 = blockIdx.y * 128;
-  const int nh = blockIdx.z;  // latent half [256 nh, +256)
+  const int nh = blockIdx.z;  // latent part [256 nh, +nw)
+  const int dc = a.d_c;
+  const int nw = dc < 256 ? dc : 256;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
   if (threadIdx.x == 0) {
@@ -116,14 +121,14 @@ absorb_tc_kernel(const __grid_constant__ CUtensorMap map_wuk, const __grid_const
     // __syncwarp so that no lane of this warp polls a barrier lane 0 has yet to release
     if (lane == 0) {
       const uint64_t stream_once = l2_policy_evict_first(), keep = l2_policy_evict_last();
-      mbar_arrive_expect_tx(&bars[0], C::Q_BYTES + C::W_BYTES);
+      mbar_arrive_expect_tx(&bars[0], C::Q_BYTES + 2 * nw * 128);
       for (int kb = 0; kb < 2; ++kb)
         tma_load_2d(qbuf + kb * 16384, &map_q, &bars[0], i * 192 + 64 * kb, s0, stream_once);
-      for (int kb = 0; kb < 2; ++kb)
-        tma_load_2d(wbuf + kb * 32768, &map_wuk, &bars[0], 64 * kb, i * 512 + 256 * nh, keep);
+      for (int kb = 0; kb < 2; ++kb)  // box {64, nw}
+        tma_load_2d(wbuf + kb * 32768, &map_wuk, &bars[0], 64 * kb, i * dc + 256 * nh, keep);
       if (mbar_wait(&bars[0], 0, kWaitNs, abort_flag, a.status, 40)) {
         tc_fence_after();
-        constexpr uint32_t idesc = idesc_bf16_f32(128, 256, false);
+        const uint32_t idesc = nw == 256 ? idesc_bf16_f32(128, 256, false) : idesc_bf16_f32(128, 128, false);
         const uint32_t qa = smem_u32(qbuf), wa = smem_u32(wbuf);
 #pragma unroll
         for (int ks = 0; ks < 8; ++ks) {
@@ -146,8 +151,8 @@ absorb_tc_kernel(const __grid_constant__ CUtensorMap map_wuk, const __grid_const
   const int r = 32 * (warp & 3) + lane;  // sequence within the chunk = TMEM lane
   const int s = s0 + r;
   const int part = warp >> 2;            // columns [256 nh + 128 part, +128); rope pairs [16 part, +16)
-  const long long lo_off = static_cast<long long>(a.batch) * a.heads * 576;
-  const long long row = (static_cast<long long>(s) * a.heads + i) * 576;
+  const long long lo_off = static_cast<long long>(a.batch) * a.heads * (dc + 64);
+  const long long row = (static_cast<long long>(s) * a.heads + i) * (dc + 64);
   if (s < a.batch && nh == 0) {
     // RoPE of the query's rope part at position L-1, while the loads and MMAs run: pair
     // (j, j + 32) turns by pos * theta^(-2j/64) radians.  The angle is carried in turns
@@ -177,7 +182,7 @@ absorb_tc_kernel(const __grid_constant__ CUtensorMap map_wuk, const __grid_const
 #pragma unroll
       for (int h2 = 0; h2 < 2; ++h2) {
         const float* y = h2 == 0 ? y1 : y2;
-        const long long dst = row + 512 + 32 * h2 + 16 * part;
+        const long long dst = row + dc + 32 * h2 + 16 * part;
 #pragma unroll
         for (int v = 0; v < 2; ++v) {
           __align__(16) __half h8[8];
@@ -190,7 +195,7 @@ absorb_tc_kernel(const __grid_constant__ CUtensorMap map_wuk, const __grid_const
   }
   const bool done = mbar_wait(&bars[1], 0, kWaitNs, abort_flag, a.status, 41);
   tc_fence_after();
-  if (done && !*abort_flag) {
+  if (done && !*abort_flag && 128 * part < nw) {
     const float scale = a.alpha_q * a.alpha_kv;
     const uint32_t lane_base = static_cast<uint32_t>(32 * (warp & 3)) << 16;
 #pragma unroll 1
@@ -217,7 +222,7 @@ absorb_tc_kernel(const __grid_constant__ CUtensorMap map_wuk, const __grid_const
 }
 
 // ---------------------------------------------------------------------------- merge
-// grid (ceil(h / (256 / TPH)), 4 slices, B), 256 * Z threads.  Thread = (head, CPT
+// grid (ceil(h / (256 / TPH)), d_c / 128 slices, B), 256 * Z threads.  Thread = (head, CPT
 // consecutive latent columns of the slice); the Z thread sets take alternate runs of GU
 // groups and are merged through shared memory at the end.  Every load of a run of GU
 // groups is issued before any of them is used.
@@ -249,7 +254,7 @@ __global__ void __launch_bounds__(256 * Z) merge_kernel(const CombineArgs a) {
         const int g = gb + u;
         // a group with an empty tile range (more groups than tiles) wrote nothing
         const bool live = g <= g_hi && group_tile_begin(g, G, T) != group_tile_begin(g + 1, G, T);
-        const long long row = ((static_cast<long long>(g) + seq) * 4 + slice) * 128 + head;
+        const long long row = ((static_cast<long long>(g) + seq) * gridDim.y + slice) * 128 + head;
         ml[u] = live ? a.ml_part[row] : make_float2(-INFINITY, 0.f);
 #pragma unroll
         for (int v = 0; v < V; ++v)
@@ -300,8 +305,8 @@ __global__ void __launch_bounds__(256 * Z) merge_kernel(const CombineArgs a) {
   }
   if (head >= a.heads) return;
   const float inv = den > 0.f ? 1.f / den : 0.f;  // an empty sequence gives zeros
-  // o_lat as hi / lo bf16 terms, [h][B][512] each
-  const long long base = (static_cast<long long>(head) * a.batch + seq) * 512 + 128 * slice + col;
+  // o_lat as hi / lo bf16 terms, [h][B][d_c] each
+  const long long base = (static_cast<long long>(head) * a.batch + seq) * a.d_c + 128 * slice + col;
   __align__(16) __nv_bfloat16 hi[CPT], lo[CPT];
 #pragma unroll
   for (int u = 0; u < CPT; ++u) {
@@ -309,7 +314,7 @@ __global__ void __launch_bounds__(256 * Z) merge_kernel(const CombineArgs a) {
     hi[u] = __float2bfloat16_rn(x);
     lo[u] = __float2bfloat16_rn(x - __bfloat162float(hi[u]));
   }
-  __nv_bfloat16* lo_base = a.o_lat + static_cast<long long>(a.heads) * a.batch * 512;
+  __nv_bfloat16* lo_base = a.o_lat + static_cast<long long>(a.heads) * a.batch * a.d_c;
   if constexpr (CPT >= 8) {
 #pragma unroll
     for (int v = 0; v < CPT / 8; ++v) {
@@ -328,8 +333,7 @@ struct UpprojCfg {
   static constexpr int A_BYTES = 2 * 2 * 128 * 128;  // hi, lo x 2 latent boxes of [128 sequences x 128 B]
   static constexpr int B_BYTES = 2 * 128 * 128;      // 2 output-column boxes of [128 latent rows x 128 B]
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
-  static constexpr int STAGES = 2;
-  static constexpr int CHUNKS = 4;                   // K chunks of 128 latent
+  static constexpr int STAGES = 2;                   // K chunks of 128 latent: d_c / 128 of them
   static constexpr int SMEM = 1024 + STAGES * STAGE_BYTES + 64;
   static constexpr int TMEM_COLS = 128;
   static constexpr int THREADS = 256;
@@ -381,12 +385,13 @@ upproj_tc_kernel(const __grid_constant__ CUtensorMap map_wuv, const __grid_const
       // only the 32-row boxes that hold this chunk's sequences are loaded; the other A
       // rows feed D rows that are never stored
       const int nbox = min(4, (a.batch - s0 + 31) / 32);
+      const int nchunks = a.d_c / 128;
       auto load_w = [&](int c) {  // W_UV rows of chunk c (an input of the call) + the byte count
         uint8_t* st = stages + (c % C::STAGES) * C::STAGE_BYTES;
         uint64_t* bar = &full[c % C::STAGES];
         mbar_arrive_expect_tx(bar, 4 * nbox * 4096 + C::B_BYTES);
         for (int db = 0; db < 2; ++db)
-          tma_load_2d(st + C::A_BYTES + db * 16384, &map_wuv, bar, 64 * db, i * 512 + 128 * c, keep);
+          tma_load_2d(st + C::A_BYTES + db * 16384, &map_wuv, bar, 64 * db, i * a.d_c + 128 * c, keep);
       };
       auto load_o = [&](int c) {  // o_lat rows of chunk c, written by the merge kernel
         uint8_t* st = stages + (c % C::STAGES) * C::STAGE_BYTES;
@@ -401,16 +406,15 @@ upproj_tc_kernel(const __grid_constant__ CUtensorMap map_wuv, const __grid_const
         load_w(c);
         load_o(c);
       };
-      load_w(0);
-      load_w(1);
+      const int first = min(C::STAGES, nchunks);  // chunks loaded before the first MMA
+      for (int c = 0; c < first; ++c) load_w(c);
       grid_dep_wait();
-      load_o(0);
-      load_o(1);
-      int issued = 2;
+      for (int c = 0; c < first; ++c) load_o(c);
+      int issued = first;
       constexpr uint32_t idesc = idesc_bf16_f32(128, 128, true);  // B (W_UV) MN-major
       const uint32_t base = smem_u32(stages);
       bool ok = true;
-      for (int c = 0; c < C::CHUNKS && ok; ++c) {
+      for (int c = 0; c < nchunks && ok; ++c) {
         const int st = c % C::STAGES;
         if (!mbar_wait(&full[st], (c / C::STAGES) & 1, kWaitNs, abort_flag, a.status, 42)) {
           ok = false;
@@ -430,7 +434,7 @@ upproj_tc_kernel(const __grid_constant__ CUtensorMap map_wuv, const __grid_const
         umma_commit(&empty[st]);
         // refill the other stage once the previous chunk's MMAs (queued ahead of these)
         // have read it
-        if (c >= 1 && c + 1 < C::CHUNKS) {
+        if (c >= 1 && c + 1 < nchunks) {
           const int prev = c - 1;
           if (!mbar_wait(&empty[prev % C::STAGES], (prev / C::STAGES) & 1, kWaitNs, abort_flag, a.status, 43)) {
             ok = false;
@@ -443,7 +447,7 @@ upproj_tc_kernel(const __grid_constant__ CUtensorMap map_wuv, const __grid_const
       umma_commit(done_bar);  // every MMA issued above (possibly none) completed
       if (!ok) {  // copies still in flight land before the CTA may exit
         volatile int never = 0;
-        for (int k = issued - C::STAGES; k < issued; ++k)
+        for (int k = max(0, issued - C::STAGES); k < issued; ++k)
           mbar_wait(&full[k % C::STAGES], (k / C::STAGES) & 1, kWaitNs, &never, a.status, 44);
       }
     }
@@ -506,7 +510,8 @@ cudaError_t launch_absorb_q(const CUtensorMap& map_wuk, const CUtensorMap& map_q
                             cudaStream_t stream, bool pdl) {
   cudaError_t e = set_smem(absorb_tc_kernel, AbsorbCfg::SMEM);
   if (e != cudaSuccess) return e;
-  return launch_kernel(absorb_tc_kernel, dim3(a.heads, (a.batch + 127) / 128, 2), dim3(AbsorbCfg::THREADS),
+  return launch_kernel(absorb_tc_kernel, dim3(a.heads, (a.batch + 127) / 128, a.d_c > 256 ? a.d_c / 256 : 1),
+                       dim3(AbsorbCfg::THREADS),
                        AbsorbCfg::SMEM, stream, pdl, map_wuk, map_q, a);
 }
 
@@ -516,9 +521,11 @@ cudaError_t launch_combine_upproj(const CUtensorMap& map_wuv, const CUtensorMap&
   // groups): 8 heads x 1 float4 per block and two thread sets over alternate group runs.
   cudaError_t e;
   if (a.batch >= 16)
-    e = launch_kernel(merge_kernel<16, 1, 2>, dim3((a.heads + 31) / 32, 4, a.batch), dim3(256), 0, stream, pdl, a);
+    e = launch_kernel(merge_kernel<16, 1, 2>, dim3((a.heads + 31) / 32, a.d_c / 128, a.batch), dim3(256), 0, stream,
+                      pdl, a);
   else
-    e = launch_kernel(merge_kernel<4, 2, 4>, dim3((a.heads + 7) / 8, 4, a.batch), dim3(512), 0, stream, pdl, a);
+    e = launch_kernel(merge_kernel<4, 2, 4>, dim3((a.heads + 7) / 8, a.d_c / 128, a.batch), dim3(512), 0, stream,
+                      pdl, a);
   if (e != cudaSuccess) return e;
   if ((e = set_smem(upproj_tc_kernel, UpprojCfg::SMEM)) != cudaSuccess) return e;
   return launch_kernel(upproj_tc_kernel, dim3(a.heads, (a.batch + 127) / 128), dim3(UpprojCfg::THREADS),

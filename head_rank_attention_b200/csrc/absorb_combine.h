@@ -12,24 +12,26 @@ namespace hra {
 struct AbsorbArgs {
   const __nv_bfloat16* q;     // [B, h, 192]
   const int32_t* seq_lens;    // [B]
-  __half* q_tilde;            // out: fp16 [B, h, 576], or (two_term) bf16 hi [B, h, 576] + bf16 lo [B, h, 576]
-  int two_term;               // 1: store q~ as bf16 hi + bf16 lo (MLRA-4 kernel); 0: fp16
+  __half* q_tilde;            // out: fp16 [B, h, d_c + 64], or (two_term) bf16 hi then bf16 lo, each [B, h, d_c + 64]
+  int two_term;               // 1: store q~ as bf16 hi + bf16 lo (128-wide-branch kernel); 0: fp16
   int* status;                // cleared by this kernel (first kernel of a call)
   int* tile_prefix;           // out: [B + 1] exclusive prefix of decode tiles per sequence
   int tile_tokens;            // decode tile size (tokens)
   int batch, heads;
+  int d_c;                    // latent width: 512, or 256 / 128 (a shard of 128-wide branches)
   float alpha_q, alpha_kv, rope_theta;
 };
 
 struct CombineArgs {
-  const float* o_part;        // [slots, 4, 128, 128]
-  const float2* ml_part;      // [slots, 4, 128]
+  const float* o_part;        // [slots, d_c / 128, 128, 128]
+  const float2* ml_part;      // [slots, d_c / 128, 128]
   const int* tile_prefix;     // [B + 1], written by the absorb kernel
-  __nv_bfloat16* o_lat;       // merged latent output, bf16 hi [h, B, 512] then bf16 lo [h, B, 512]
+  __nv_bfloat16* o_lat;       // merged latent output, bf16 hi [h, B, d_c] then bf16 lo [h, B, d_c]
   int* status;                // device status word (expired waits)
   float* out_f32;             // [B, h, 128] or nullptr
   __nv_bfloat16* out_bf16;    // [B, h, 128] or nullptr
   int batch, heads, groups;
+  int d_c;                    // latent width (as in AbsorbArgs)
   float alpha_kv, branch_scale;
 };
 
@@ -38,13 +40,13 @@ int absorb_seq_chunk(int batch);
 // Rows of one o_lat box in the up-projection (its CTAs take 128 sequences in boxes of this many).
 int upproj_seq_chunk();
 
-// map_wuk: W_UK viewed as [h*512 rows, 128] bf16, box {64, 256}, SWIZZLE_128B.
+// map_wuk: W_UK viewed as [h*d_c rows, 128] bf16, box {64, min(d_c, 256)}, SWIZZLE_128B.
 // map_q:   q viewed as [B rows, h*192] bf16, box {64, absorb_seq_chunk(B)}, SWIZZLE_128B.
 // pdl: launch with programmatic dependent launch (launch.h).
 cudaError_t launch_absorb_q(const CUtensorMap& map_wuk, const CUtensorMap& map_q, const AbsorbArgs& a,
                             cudaStream_t stream, bool pdl);
-// map_wuv:  W_UV viewed as [h*512 rows, 128] bf16, box {64, 128}, SWIZZLE_128B.
-// map_olat: a.o_lat viewed as [2*h*B rows, 512] bf16, box {64, upproj_seq_chunk()}, SWIZZLE_128B.
+// map_wuv:  W_UV viewed as [h*d_c rows, 128] bf16, box {64, 128}, SWIZZLE_128B.
+// map_olat: a.o_lat viewed as [2*h*B rows, d_c] bf16, box {64, upproj_seq_chunk()}, SWIZZLE_128B.
 cudaError_t launch_combine_upproj(const CUtensorMap& map_wuv, const CUtensorMap& map_olat, const CombineArgs& a,
                                   cudaStream_t stream, bool pdl);
 

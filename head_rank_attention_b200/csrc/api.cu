@@ -59,11 +59,19 @@ hra_status sm_count(int* n) {
 
 hra_status validate(const hra_decode_params* p) {
   if (p == nullptr) return fail(HRA_ERR_INVALID_ARG, "params is NULL");
-  if (p->d_c != 512 || p->d_rope != 64 || p->d_nope != 128 || p->d_v != 128)
-    return fail(HRA_ERR_UNSUPPORTED, "widths (d_c=%d, d_rope=%d, d_nope=%d, d_v=%d) must be 512/64/128/128",
-                p->d_c, p->d_rope, p->d_nope, p->d_v);
-  if (p->n_branch != 1 && p->n_branch != 2 && p->n_branch != 4)
-    return fail(HRA_ERR_UNSUPPORTED, "n_branch=%d (supported: 1, 2, 4)", p->n_branch);
+  if (p->d_rope != 64 || p->d_nope != 128 || p->d_v != 128)
+    return fail(HRA_ERR_UNSUPPORTED, "widths (d_rope=%d, d_nope=%d, d_v=%d) must be 64/128/128", p->d_rope,
+                p->d_nope, p->d_v);
+  if (p->d_c == 512) {
+    if (p->n_branch != 1 && p->n_branch != 2 && p->n_branch != 4)
+      return fail(HRA_ERR_UNSUPPORTED, "n_branch=%d (supported with d_c=512: 1, 2, 4)", p->n_branch);
+  } else if (!((p->d_c == 128 || p->d_c == 256) && p->d_c == 128 * p->n_branch)) {
+    // a shard of 128-wide branches: d_c = 128 * (branches held)
+    return fail(HRA_ERR_UNSUPPORTED,
+                "d_c=%d with n_branch=%d (supported: d_c=512 with n_branch 1, 2, 4; or a shard of 128-wide "
+                "branches, d_c = 128 * n_branch = 128 or 256)",
+                p->d_c, p->n_branch);
+  }
   if (p->batch < 1 || p->batch > hra::kMaxBatch)
     return fail(HRA_ERR_UNSUPPORTED, "batch=%d (supported: 1..%d)", p->batch, hra::kMaxBatch);
   if (p->num_heads < 1 || p->num_heads > 128)
@@ -75,8 +83,9 @@ hra_status validate(const hra_decode_params* p) {
     if (x.ptr == nullptr) return fail(HRA_ERR_INVALID_ARG, "%s is NULL", x.name);
     if (!aligned16(x.ptr)) return fail(HRA_ERR_INVALID_ARG, "%s is not 16-byte aligned", x.name);
   }
-  if (p->ckv_stride < 512 || p->ckv_stride % 8 != 0)
-    return fail(HRA_ERR_INVALID_ARG, "ckv_stride=%lld must be >= 512 and a multiple of 8", (long long)p->ckv_stride);
+  if (p->ckv_stride < p->d_c || p->ckv_stride % 8 != 0)
+    return fail(HRA_ERR_INVALID_ARG, "ckv_stride=%lld must be >= d_c=%d and a multiple of 8",
+                (long long)p->ckv_stride, p->d_c);
   if (p->krope_stride < 64 || p->krope_stride % 8 != 0)
     return fail(HRA_ERR_INVALID_ARG, "krope_stride=%lld must be >= 64 and a multiple of 8",
                 (long long)p->krope_stride);
@@ -106,19 +115,20 @@ hra_status make_plan(const hra_decode_params* p, Plan* plan) {
   } else {
     hra_status st = sm_count(&sms);
     if (st != HRA_OK) return st;
-    plan->groups = sms / 4 > 0 ? sms / 4 : 1;
+    plan->groups = sms / (p->d_c / 128) > 0 ? sms / (p->d_c / 128) : 1;  // one CTA per SM
   }
   if (plan->groups > 65535) return fail(HRA_ERR_INVALID_ARG, "num_splits=%d too large", plan->groups);
   plan->slots = static_cast<long long>(plan->groups) + p->batch;
+  const size_t slices = static_cast<size_t>(p->d_c) / 128;
   size_t off = 256;  // device status word
-  plan->q_tilde = off;
-  off = round256(off + 2 * static_cast<size_t>(p->batch) * p->num_heads * 576 * sizeof(__half));  // up to two terms
+  plan->q_tilde = off;  // up to two terms of [B, h, d_c + 64]
+  off = round256(off + 2 * static_cast<size_t>(p->batch) * p->num_heads * (p->d_c + 64) * sizeof(__half));
   plan->o_part = off;
-  off = round256(off + static_cast<size_t>(plan->slots) * 4 * 128 * 128 * sizeof(float));
+  off = round256(off + static_cast<size_t>(plan->slots) * slices * 128 * 128 * sizeof(float));
   plan->ml_part = off;
-  off = round256(off + static_cast<size_t>(plan->slots) * 4 * 128 * sizeof(float2));
+  off = round256(off + static_cast<size_t>(plan->slots) * slices * 128 * sizeof(float2));
   plan->o_lat = off;  // merged latent output as two bf16 terms
-  off = round256(off + 2 * static_cast<size_t>(p->num_heads) * p->batch * 512 * sizeof(__nv_bfloat16));
+  off = round256(off + 2 * static_cast<size_t>(p->num_heads) * p->batch * p->d_c * sizeof(__nv_bfloat16));
   plan->tile_prefix = off;  // decode tiles per sequence, exclusive prefix [B + 1]
   off = round256(off + (static_cast<size_t>(p->batch) + 1) * sizeof(int));
   plan->total = off;
@@ -172,17 +182,18 @@ hra_status run_decode(const hra_decode_params* p, cudaStream_t stream) {
 
   // Every tensor map is encoded before the first launch so that no host work sits between
   // the kernels of one call.
-  const int h = p->num_heads, B = p->batch;
+  const int h = p->num_heads, B = p->batch, dc = p->d_c;
   CUtensorMap map_wuk, map_q, map_wuv, map_olat, map_ckv, map_krope;
-  if ((st = encode_map(&map_wuk, p->w_uk, 128, static_cast<int64_t>(h) * 512, 128, 256)) != HRA_OK) return st;
+  if ((st = encode_map(&map_wuk, p->w_uk, 128, static_cast<int64_t>(h) * dc, 128, dc < 256 ? dc : 256)) != HRA_OK)
+    return st;
   if ((st = encode_map(&map_q, p->q, static_cast<int64_t>(h) * 192, B, static_cast<int64_t>(h) * 192,
                        hra::absorb_seq_chunk(B))) != HRA_OK)
     return st;
-  if ((st = encode_map(&map_wuv, p->w_uv, 128, static_cast<int64_t>(h) * 512, 128, 128)) != HRA_OK) return st;
-  if ((st = encode_map(&map_olat, o_lat, 512, 2 * static_cast<int64_t>(h) * B, 512, hra::upproj_seq_chunk())) !=
+  if ((st = encode_map(&map_wuv, p->w_uv, 128, static_cast<int64_t>(h) * dc, 128, 128)) != HRA_OK) return st;
+  if ((st = encode_map(&map_olat, o_lat, dc, 2 * static_cast<int64_t>(h) * B, dc, hra::upproj_seq_chunk())) !=
       HRA_OK)
     return st;
-  if ((st = encode_map(&map_ckv, p->ckv, 512, p->cache_rows, p->ckv_stride, 32)) != HRA_OK) return st;
+  if ((st = encode_map(&map_ckv, p->ckv, dc, p->cache_rows, p->ckv_stride, 32)) != HRA_OK) return st;
   if ((st = encode_map(&map_krope, p->krope, 64, p->cache_rows, p->krope_stride, 32)) != HRA_OK) return st;
 
   auto mark = [&](int k) -> cudaError_t {
@@ -201,9 +212,10 @@ hra_status run_decode(const hra_decode_params* p, cudaStream_t stream) {
   ab.alpha_q = p->alpha_q;
   ab.alpha_kv = p->alpha_kv;
   ab.rope_theta = p->rope_theta;
-  ab.two_term = p->n_branch == 4 ? 1 : 0;
+  ab.d_c = dc;
+  ab.two_term = dc / p->n_branch == 128 ? 1 : 0;  // 128-wide branches: the two-term split kernel
   ab.tile_prefix = tile_prefix;
-  ab.tile_tokens = hra::decode_tile_tokens(p->n_branch);
+  ab.tile_tokens = hra::decode_tile_tokens(dc / p->n_branch);
   // Programmatic dependent launch lets each kernel start while the previous one drains;
   // the stage-timing mode launches plainly so that its events bracket whole kernels.
   const bool pdl = p->stage_events == nullptr;
@@ -221,6 +233,7 @@ hra_status run_decode(const hra_decode_params* p, cudaStream_t stream) {
   da.cache_rows = p->cache_rows;
   da.batch = p->batch;
   da.heads = p->num_heads;
+  da.d_c = dc;
   da.scale_log2 = tau * 1.4426950408889634f;
   da.o_part = o_part;
   da.ml_part = ml_part;
@@ -242,6 +255,7 @@ hra_status run_decode(const hra_decode_params* p, cudaStream_t stream) {
   cb.batch = p->batch;
   cb.heads = p->num_heads;
   cb.groups = plan.groups;
+  cb.d_c = dc;
   cb.alpha_kv = p->alpha_kv;
   cb.branch_scale = p->branch_scale;
   e = hra::launch_combine_upproj(map_wuv, map_olat, cb, stream, pdl);

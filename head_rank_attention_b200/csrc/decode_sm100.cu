@@ -488,12 +488,16 @@ cudaError_t launch_decode(const CUtensorMap& map_ckv, const CUtensorMap& map_kro
 
 }  // namespace
 
-int decode_tile_tokens(int n_branch) { return n_branch == 4 ? decode_split_tile_tokens() : (n_branch == 2 ? 64 : 32); }
+int decode_tile_tokens(int branch_width) {
+  return branch_width == 128 ? decode_split_tile_tokens() : (branch_width == 256 ? 64 : 32);
+}
 
 cudaError_t launch_decode_kernel(int n_branch, const CUtensorMap& map_ckv, const CUtensorMap& map_krope,
                                  const DecodeArgs& a, int groups, cudaStream_t stream, bool pdl) {
+  if (n_branch < 1 || a.d_c % n_branch != 0) return cudaErrorInvalidValue;
+  if (a.d_c / n_branch == 128) return launch_decode_split_kernel(map_ckv, map_krope, a, groups, stream, pdl);
+  if (a.d_c != 512) return cudaErrorInvalidValue;  // this kernel assumes the whole 512-wide latent
   switch (n_branch) {
-    case 4: return launch_decode_split_kernel(map_ckv, map_krope, a, groups, stream, pdl);
     case 2: return launch_decode<2, 64, 5>(map_ckv, map_krope, a, groups, stream, pdl);
     case 1: return launch_decode<1, 32, 5>(map_ckv, map_krope, a, groups, stream, pdl);
     default: return cudaErrorInvalidValue;

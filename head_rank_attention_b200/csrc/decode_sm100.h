@@ -10,9 +10,9 @@ namespace hra {
 
 // Arguments of one decode launch (device pointers; see hra.h for layouts).
 struct DecodeArgs {
-  const __half* q_tilde;      // absorbed latent query (512) | rotated rope (64) per (sequence, head):
-                              //   fp16 [B, h, 576], or for the MLRA-4 kernel bf16 hi [B, h, 576]
-                              //   followed by bf16 lo [B, h, 576]
+  const __half* q_tilde;      // absorbed latent query (d_c) | rotated rope (64) per (sequence, head):
+                              //   fp16 [B, h, d_c + 64], or for the 128-wide-branch kernel bf16 hi
+                              //   [B, h, d_c + 64] followed by bf16 lo [B, h, d_c + 64]
   const int32_t* seq_lens;    // int32 [B]
   const int32_t* block_table; // int32 [B, max_pages] or nullptr (contiguous layout)
   int max_pages;
@@ -21,9 +21,10 @@ struct DecodeArgs {
   long long cache_rows;       // rows addressable through the tensor maps
   int batch;
   int heads;
+  int d_c;                    // latent width held by this call: 512, or 256 / 128 for a branch shard
   float scale_log2;           // softmax scale * log2(e)
-  float* o_part;              // fp32 [slots, 4, 128, 128]: un-normalised O per segment and slice
-  float2* ml_part;            // fp32 [slots, 4, 128] pairs: (running max in log2 units, row sum)
+  float* o_part;              // fp32 [slots, d_c / 128, 128, 128]: un-normalised O per segment and slice
+  float2* ml_part;            // fp32 [slots, d_c / 128, 128] pairs: (running max in log2 units, row sum)
   int* status;                // device status word
   uint64_t wait_limit_ns;     // global-time budget of one device-side wait
 };
@@ -50,16 +51,18 @@ __device__ __forceinline__ int cache_chunk_row(const DecodeArgs& a, int s, int t
   return static_cast<int>(row);
 }
 
-// Tokens per cache tile for a branch count (decides the TMEM and shared-memory budget).
-int decode_tile_tokens(int n_branch);
+// Tokens per cache tile for a branch width (decides the TMEM and shared-memory budget).
+int decode_tile_tokens(int branch_width);
 int decode_split_tile_tokens();
 
-// MLRA-4 kernel on the bf16 cache with a two-term bf16 query (grid: 4 branches x groups).
+// 128-wide-branch kernel (MLRA-4, or a shard of its branches) on the bf16 cache with a
+// two-term bf16 query; grid (d_c / 128 branches, groups).
 cudaError_t launch_decode_split_kernel(const CUtensorMap& map_ckv, const CUtensorMap& map_krope,
                                        const DecodeArgs& a, int groups, cudaStream_t stream, bool pdl);
 
-// Launch the decode kernel on grid (4 slices, `groups` KV splits); pdl: programmatic
-// dependent launch (launch.h).
+// Launch the decode kernel on grid (d_c / 128 slices, `groups` KV splits); pdl:
+// programmatic dependent launch (launch.h).  Branches 128 wide run the split kernel, 256
+// and 512 wide (d_c = 512 only) the converting kernel.
 cudaError_t launch_decode_kernel(int n_branch, const CUtensorMap& map_ckv, const CUtensorMap& map_krope,
                                  const DecodeArgs& a, int groups, cudaStream_t stream, bool pdl);
 

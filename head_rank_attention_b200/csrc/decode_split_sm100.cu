@@ -3,7 +3,8 @@
 //
 // Same computation and work decomposition as decode_sm100.cu (step 2 of "Multi-Head
 // Low-Rank Attention", 方法步骤详情; one CTA per 128-wide latent slice = one MLRA-4
-// branch, groups of 4 CTAs over contiguous tile ranges), but the latent part of the
+// branch, groups of d_c / 128 CTAs over contiguous tile ranges: 4 for MLRA-4, fewer when
+// the call holds a shard of the branches), but the latent part of the
 // cache tile is never rewritten: the absorbed query is carried as two bf16 terms
 // q~ = q_hi + q_lo (q_lo = bf16(q~ - q_hi), together ~16 significant bits), and every
 // latent score is the fp32 sum of two bf16 MMAs against the same bf16 tile.  The rope
@@ -346,7 +347,8 @@ decode_split_kernel(const __grid_constant__ CUtensorMap map_ckv, const __grid_co
     const uint32_t t_row = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
     const float sl2 = a.scale_log2;
     const __nv_bfloat16* q_hi = reinterpret_cast<const __nv_bfloat16*>(a.q_tilde);
-    const __nv_bfloat16* q_lo = q_hi + static_cast<long long>(a.batch) * a.heads * 576;
+    const int q_stride = a.d_c + 64;  // query row: d_c latent columns then the rope part
+    const __nv_bfloat16* q_lo = q_hi + static_cast<long long>(a.batch) * a.heads * q_stride;
     TileCursor cur;
     cur.init(prefix, B, t_begin, t_end, s_first);
     int it = 0, seg = 0;
@@ -354,16 +356,16 @@ decode_split_kernel(const __grid_constant__ CUtensorMap map_ckv, const __grid_co
     while (ok && cur.valid) {
       const int s = cur.s;
       const int L = a.seq_lens[s];
-      // this head's query for the branch: latent columns [128 slice, +128) then rope [512, 576);
+      // this head's query for the branch: latent columns [128 slice, +128) then rope [d_c, d_c + 64);
       // half 0 stores q_hi, half 1 stores q_lo
       {
-        const long long base = (static_cast<long long>(s) * a.heads + min(row, a.heads - 1)) * 576;
+        const long long base = (static_cast<long long>(s) * a.heads + min(row, a.heads - 1)) * q_stride;
         const bool live = row < a.heads;
         const uint4* src = reinterpret_cast<const uint4*>((half == 0 ? q_hi : q_lo) + base);
         const uint32_t col = half == 0 ? C::TMEM_QH : C::TMEM_QL;
 #pragma unroll 1
         for (int c = 0; c < 2 + (half == 0); ++c) {  // latent chunks, then (half 0) the fp16 rope
-          const int e0 = c < 2 ? slice * 128 + 64 * c : 512;  // 16-bit element
+          const int e0 = c < 2 ? slice * 128 + 64 * c : a.d_c;  // 16-bit element
           uint32_t w[32];
 #pragma unroll
           for (int u = 0; u < 8; ++u) {
@@ -461,7 +463,8 @@ decode_split_kernel(const __grid_constant__ CUtensorMap map_ckv, const __grid_co
       if (!warp_wait(pv_done, (it - 1) & 1, limit, abort_flag, status, 32)) { ok = false; break; }
       tc_fence_after();
       const long long slot = static_cast<long long>(g) + s;
-      float4* dst = reinterpret_cast<float4*>(a.o_part + ((slot * 4 + slice) * 128 + row) * 128 + 64 * half);
+      float4* dst =
+          reinterpret_cast<float4*>(a.o_part + ((slot * gridDim.x + slice) * 128 + row) * 128 + 64 * half);
 #pragma unroll 1
       for (int k = 0; k < 2; ++k) {
         uint32_t o[32];
@@ -480,7 +483,7 @@ decode_split_kernel(const __grid_constant__ CUtensorMap map_ckv, const __grid_co
       if (!warp_wait(lsum_bar, seg & 1, limit, abort_flag, status, 34)) { ok = false; break; }
       ++seg;
       if (half == 0 && row < a.heads)
-        a.ml_part[(slot * 4 + slice) * 128 + row] = make_float2(m_ref, l + red_l[128 + row]);
+        a.ml_part[(slot * gridDim.x + slice) * 128 + row] = make_float2(m_ref, l + red_l[128 + row]);
       tc_fence_before();
     }
   }
@@ -503,7 +506,8 @@ cudaError_t launch_decode_split_kernel(const CUtensorMap& map_ckv, const CUtenso
   auto kern = decode_split_kernel<kNT, kStages>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
   if (e != cudaSuccess) return e;
-  return launch_kernel(kern, dim3(4, groups), dim3(C::THREADS), C::SMEM_BYTES, stream, pdl, map_ckv, map_krope, a);
+  return launch_kernel(kern, dim3(a.d_c / 128, groups), dim3(C::THREADS), C::SMEM_BYTES, stream, pdl, map_ckv,
+                       map_krope, a);
 }
 
 }  // namespace hra

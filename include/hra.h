@@ -13,6 +13,11 @@
  * n_branch = 1 is MLA ("ML Revisit: Attention", Multi-Head Latent Attention: the
  * absorbed QK^T = C_q W_q W_k^T C_kv^T with a decoupled RoPE key shared by all heads);
  * n_branch = 4 is MLRA-4 (核心方法: O = sum_b Softmax(Q K_b^T) V_b).
+ * Branch shards (核心方法: under 4-way tensor parallelism each device holds one MLRA-4
+ * branch's latent columns, a copy of K_RoPE and that branch's W_UK / W_UV rows): a call with
+ * d_c = 128 * n_branch in {128, 256} computes the branches it holds, and its out is that
+ * shard's part of the branch sum; summing out over the shards (an all-reduce across the
+ * devices) gives the MLRA-4 output.  Pass the full model's branch_scale (1/2 for MLRA-4).
  * The softmax scale of every branch is 1/sqrt(d_nope + d_rope) by default
  * ("vllbc02MLA", DeepseekV2Attention.__init__: scaling = qk_head_dim ** -0.5).
  *
@@ -23,7 +28,8 @@
  * Bounded device waits that expire write a status word in the workspace, read back
  * by hra_check_device_status().
  * Numerics: bf16 inputs, fp32 accumulation; softmax, combine and up-projection in fp32.
- * n_branch = 4: the tensor cores read the latent part of the cache as stored, against
+ * 128-wide branches (n_branch = 4, and branch shards): the tensor cores read the latent
+ * part of the cache as stored, against
  * the absorbed query carried as two bf16 terms (hi + lo, ~16 significant bits); the rope
  * part (query and K_RoPE tile) is scored in fp16, so |K_RoPE values| must stay below 65504.
  * n_branch = 1, 2: the cache tile is converted to fp16 in shared memory and the query is
@@ -61,21 +67,24 @@ typedef enum { HRA_BF16 = 0, HRA_F32 = 1 } hra_dtype;
 
 /*
  * Parameters of one decode step.  All pointers are device pointers, 16-byte aligned.
- * Supported set: d_c = 512, d_rope = 64, d_nope = 128, d_v = 128, n_branch in {1,2,4},
- * 1 <= num_heads <= 128, 1 <= batch <= 1024.
+ * Supported set: d_rope = 64, d_nope = 128, d_v = 128; d_c = 512 with n_branch in {1,2,4},
+ * or a branch shard d_c = 128 * n_branch in {128, 256}; 1 <= num_heads <= 128,
+ * 1 <= batch <= 1024.
  */
 typedef struct {
   int batch;            /* B, number of sequences (one query token each)               */
   int num_heads;        /* h, query heads sharing the latent cache                     */
-  int n_branch;         /* 1 = MLA, 2 = two-branch MLRA, 4 = MLRA-4                     */
-  int d_c, d_rope, d_nope, d_v;   /* 512, 64, 128, 128                                  */
+  int n_branch;         /* 1 = MLA, 2 = two-branch MLRA, 4 = MLRA-4; for a branch shard,
+                           the number of 128-wide branches this call holds               */
+  int d_c, d_rope, d_nope, d_v;   /* 512 (128 or 256 for a shard), 64, 128, 128         */
 
   const void* q;        /* bf16 [B, h, d_nope + d_rope], dense: q_nope | q_rope; q_rope is
                            NOT rotated (the library rotates it at position seq_lens[b]-1) */
   const void* ckv;      /* bf16 latent rows: row r is C_KV at ckv + r * ckv_stride          */
   const void* krope;    /* bf16 RoPE-key rows, already rotated at their own positions:
                            row r at krope + r * krope_stride.  A fused [rows, 576] cache
-                           is ckv = base, krope = base + 512, both strides 576            */
+                           is ckv = base, krope = base + 512, both strides 576 (a shard's
+                           [rows, d_c + 64]: krope = base + d_c, strides d_c + 64)        */
   int64_t ckv_stride;   /* elements between consecutive rows; multiple of 8              */
   int64_t krope_stride; /* elements between consecutive rows; multiple of 8              */
   int64_t cache_rows;   /* rows addressable from ckv / krope (bounds every row access)   */
@@ -102,8 +111,8 @@ typedef struct {
 
   void* workspace;      /* scratch of at least hra_workspace_size(p) bytes, 256-B aligned */
   size_t workspace_bytes;
-  int num_splits;       /* KV splits = groups of 4 CTAs streaming disjoint token ranges;
-                           0 = one group per 4 SMs of the current device                 */
+  int num_splits;       /* KV splits = groups of d_c/128 CTAs streaming disjoint token
+                           ranges; 0 = one group per d_c/128 SMs of the current device    */
   int wait_limit;       /* microseconds one device-side wait may last; 0 = 1 s           */
   void* const* stage_events; /* optional, NULL = none: 4 caller-owned cudaEvent_t recorded on
                                 `stream` before absorption, before the split-KV decode, before
@@ -114,7 +123,8 @@ typedef struct {
  * Depends on batch, num_splits and the current device's SM count. */
 HRA_API size_t hra_workspace_size(const hra_decode_params* p);
 
-/* MLRA decode ("Multi-Head Low-Rank Attention", 方法步骤详情), n_branch in {1,2,4}. */
+/* MLRA decode ("Multi-Head Low-Rank Attention", 方法步骤详情), n_branch in {1,2,4}, or a
+ * branch shard (see above). */
 HRA_API hra_status mlra_decode(const hra_decode_params* p, void* stream /* cudaStream_t */);
 
 /* MLA decode: the same call restricted to n_branch == 1 ("ML Revisit: Attention",

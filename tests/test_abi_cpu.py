@@ -66,15 +66,16 @@ def _fake_params(**over):
     return p
 
 
-def test_workspace_size_formula():
-    p = _fake_params()
+@pytest.mark.parametrize("d_c,n_branch,splits", [(512, 4, 37), (512, 1, 37), (256, 2, 74), (128, 1, 148)])
+def test_workspace_size_formula(d_c, n_branch, splits):
+    p = _fake_params(d_c=d_c, n_branch=n_branch, num_splits=splits, ckv_stride=d_c + 64, krope_stride=d_c + 64)
     n = hra.workspace_size(p)
-    slots = 37 + 2
+    slots, slices = splits + 2, d_c // 128
     expect = 256
-    expect = -(-(expect + 2 * 2 * 128 * 576 * 2) // 256) * 256  # q~ as up to two 16-bit terms
-    expect = -(-(expect + slots * 4 * 128 * 128 * 4) // 256) * 256
-    expect = -(-(expect + slots * 4 * 128 * 8) // 256) * 256
-    expect = -(-(expect + 2 * 128 * 2 * 512 * 2) // 256) * 256  # merged latent as two bf16 terms
+    expect = -(-(expect + 2 * 2 * 128 * (d_c + 64) * 2) // 256) * 256  # q~ as up to two 16-bit terms
+    expect = -(-(expect + slots * slices * 128 * 128 * 4) // 256) * 256
+    expect = -(-(expect + slots * slices * 128 * 8) // 256) * 256
+    expect = -(-(expect + 2 * 128 * 2 * d_c * 2) // 256) * 256  # merged latent as two bf16 terms
     expect = -(-(expect + (2 + 1) * 4) // 256) * 256  # tile prefix per sequence
     assert n == expect
 
@@ -84,6 +85,10 @@ def test_workspace_size_formula():
     (dict(ckv=0x20008), B.HRA_ERR_INVALID_ARG),          # misaligned
     (dict(n_branch=3), B.HRA_ERR_UNSUPPORTED),
     (dict(d_c=256), B.HRA_ERR_UNSUPPORTED),
+    (dict(d_c=256, n_branch=1, ckv_stride=320), B.HRA_ERR_UNSUPPORTED),   # a 256-wide branch shard
+    (dict(d_c=128, n_branch=2, ckv_stride=192), B.HRA_ERR_UNSUPPORTED),   # 64-wide branches
+    (dict(d_c=384, n_branch=3, ckv_stride=448), B.HRA_ERR_UNSUPPORTED),
+    (dict(d_c=128, n_branch=1, ckv_stride=120), B.HRA_ERR_INVALID_ARG),   # stride below d_c
     (dict(num_heads=129), B.HRA_ERR_UNSUPPORTED),
     (dict(batch=0), B.HRA_ERR_UNSUPPORTED),
     (dict(ckv_stride=580), B.HRA_ERR_INVALID_ARG),        # not a multiple of 8

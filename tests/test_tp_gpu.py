@@ -1,0 +1,93 @@
+"""GPU parity of branch shards (tensor parallelism by branch, "Multi-Head Low-Rank
+Attention", 核心方法: under 4-way TP each device holds one MLRA-4 branch).
+
+Every rank of a 2- or 4-way split runs here in turn on the one GPU: each call holds its
+shard of the cache (its 128-wide branches + K_RoPE, laid out by head_rank_attention_b200.tp)
+and of W_UK / W_UV, and the shard outputs are summed on the device as the all-reduce
+would.  Each shard is compared with the oracle on the same shard, and the sum with the
+oracle's MLRA-4 output, under the parity bar.
+"""
+import numpy as np
+import pytest
+import torch
+
+import head_rank_attention_b200 as hra
+from head_rank_attention_b200 import tp
+import oracle
+import synth
+from gpu_cases import assert_parity
+
+pytestmark = pytest.mark.gpu
+
+
+def _wl(name, lengths, heads=128, page_size=0, **kw):
+    return synth.Workload(name, 4, len(lengths), heads, max(lengths), page_size=page_size,
+                          lengths=tuple(lengths), **kw)
+
+
+CASES = [
+    (_wl("tails", (1, 31, 32, 33, 127, 128, 129, 1000)), 4, 0),
+    (_wl("tails", (1, 31, 32, 33, 127, 128, 129, 1000)), 2, 0),
+    (_wl("paged64", (5, 64, 65, 700), page_size=64), 4, 0),
+    (_wl("paged32", (5, 64, 65, 700), page_size=32), 2, 0),
+    (_wl("h16", (2048,), heads=16, alpha_q=2048 ** 0.5 / 1536 ** 0.5, alpha_kv=2.0, branch_scale=0.5), 4, 0),
+    (_wl("stress", (3000, 17), alpha_q=synth.A_Q_V3, alpha_kv=synth.A_KV_V3), 4, 0),
+    (_wl("splits1", (1, 130, 2000, 64)), 4, 1),
+    (_wl("splits200", (1, 130, 2000, 64)), 2, 200),
+]
+
+
+def _run_shard(dev, wl, rank, world, num_splits):
+    local = tp.shard_cache(dev.cache, rank, world)
+    w_uk, w_uv = tp.shard_weights(dev.w_uk, dev.w_uv, rank, world)
+    d = local.shape[1] - synth.D_ROPE
+    out = torch.empty(wl.batch, wl.heads, synth.D_V, dtype=torch.float32, device="cuda")
+    p = hra.make_params(dev.q, local[:, :d], local[:, d:], dev.seq_lens, w_uk, w_uv, out,
+                        n_branch=4 // world, alpha_q=wl.alpha_q, alpha_kv=wl.alpha_kv,
+                        branch_scale=wl.sigma_o, softmax_scale=wl.softmax_scale, rope_theta=wl.rope_theta,
+                        block_table=dev.block_table, page_size=wl.page_size, seq_stride=dev.seq_stride,
+                        num_splits=num_splits)
+    assert p.d_c == d == 512 // world
+    ws = hra.alloc_workspace(p)
+    ws.fill_(0xFF)  # NaN bytes: a read of a slot the call did not write shows up
+    hra.mlra_decode(p)
+    hra.check_device_status(p)
+    return out
+
+
+def _shard_ref(inp, wl, rank, world, seqs=None):
+    w_uk, w_uv = tp.shard_weights(inp.w_uk, inp.w_uv, rank, world)
+    res = []
+    for s in range(wl.batch) if seqs is None else seqs:
+        local = tp.shard_cache(synth.logical_rows(inp, wl, s), rank, world)
+        d = local.shape[1] - synth.D_ROPE
+        res.append(oracle.mlra_decode_absorbed(inp.q[s], local[:, :d], local[:, d:], w_uk, w_uv, 4 // world,
+                                               alpha_q=wl.alpha_q, alpha_kv=wl.alpha_kv, branch_scale=wl.sigma_o,
+                                               softmax_scale=wl.softmax_scale, rope_theta=wl.rope_theta))
+    return np.stack(res)
+
+
+@pytest.mark.parametrize("wl,world,num_splits", CASES,
+                         ids=[f"{c[0].name}-tp{c[1]}-splits{c[2]}" for c in CASES])
+def test_branch_shards_match_the_oracle_and_sum_to_mlra4(wl, world, num_splits):
+    inp = synth.make_inputs(wl)
+    dev = synth.to_device(inp)
+    total = torch.zeros(wl.batch, wl.heads, synth.D_V, dtype=torch.float32, device="cuda")
+    for r in range(world):
+        out = _run_shard(dev, wl, r, world, num_splits)
+        assert_parity(out.cpu().numpy(), _shard_ref(inp, wl, r, world), f"{wl.name} shard {r}/{world}")
+        total += out
+    ref = oracle.decode_batch(inp, wl, form="absorbed")
+    assert_parity(total.cpu().numpy(), ref, f"{wl.name} sum of {world} shards")
+
+
+def test_zero_length_sequence_gives_zero_row_in_every_shard():
+    wl = _wl("zero", (0, 300, 0, 33))
+    inp = synth.make_inputs(wl)
+    dev = synth.to_device(inp)
+    for world in (4, 2):
+        for r in range(world):
+            out = _run_shard(dev, wl, r, world, 0).cpu()
+            assert (out[0] == 0).all() and (out[2] == 0).all()
+            assert_parity(out[[1, 3]].numpy(), _shard_ref(inp, wl, r, world, seqs=[1, 3]),
+                          f"zero-length neighbours, shard {r}/{world}")
