@@ -91,3 +91,52 @@ def test_zero_length_sequence_gives_zero_row_in_every_shard():
             assert (out[0] == 0).all() and (out[2] == 0).all()
             assert_parity(out[[1, 3]].numpy(), _shard_ref(inp, wl, r, world, seqs=[1, 3]),
                           f"zero-length neighbours, shard {r}/{world}")
+
+
+def test_shard_bf16_output():
+    wl = _wl("bf16", (700, 33))
+    inp = synth.make_inputs(wl)
+    dev = synth.to_device(inp)
+    local = tp.shard_cache(dev.cache, 3, 4)
+    w_uk, w_uv = tp.shard_weights(dev.w_uk, dev.w_uv, 3, 4)
+    out = torch.empty(wl.batch, wl.heads, synth.D_V, dtype=torch.bfloat16, device="cuda")
+    p = hra.make_params(dev.q, local[:, :128], local[:, 128:], dev.seq_lens, w_uk, w_uv, out, n_branch=1,
+                        branch_scale=wl.sigma_o, seq_stride=dev.seq_stride)
+    ws = hra.alloc_workspace(p)
+    hra.mlra_decode(p)
+    hra.check_device_status(p)
+    assert_parity(out.float().cpu().numpy(), _shard_ref(inp, wl, 3, 4), "bf16 out, shard 3/4")
+    del ws
+
+
+def test_shard_graph_replay_and_determinism():
+    """A shard call replayed from a CUDA graph, and called again directly, gives the same bits."""
+    wl = _wl("graph", (1500, 40))
+    dev = synth.to_device(synth.make_inputs(wl))
+    ref = _run_shard(dev, wl, 1, 4, 0)
+    assert torch.equal(_run_shard(dev, wl, 1, 4, 0), ref)
+    local = tp.shard_cache(dev.cache, 1, 4)
+    w_uk, w_uv = tp.shard_weights(dev.w_uk, dev.w_uv, 1, 4)
+    out = torch.zeros_like(ref)
+    p = hra.make_params(dev.q, local[:, :128], local[:, 128:], dev.seq_lens, w_uk, w_uv, out, n_branch=1,
+                        branch_scale=wl.sigma_o, seq_stride=dev.seq_stride)
+    ws = hra.alloc_workspace(p)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        hra.mlra_decode(p, torch.cuda.current_stream())
+    for _ in range(3):
+        out.zero_()
+        g.replay()
+        torch.cuda.synchronize()
+        assert torch.equal(out, ref)
+    hra.check_device_status(p)
+    del g, ws
+
+
+def test_shard_paged_equals_contiguous_bitwise():
+    lens = (100, 640, 33)
+    outs = []
+    for page_size in (0, 32):
+        wl = _wl("layout", lens, page_size=page_size)
+        outs.append(_run_shard(synth.to_device(synth.make_inputs(wl)), wl, 2, 4, 0))
+    assert torch.equal(outs[0], outs[1])
