@@ -3,7 +3,7 @@
 //
 // The batch's cached tokens are cut into tiles of NT tokens per sequence
 // (ceil(L_s / NT) tiles for sequence s) and the tiles of all sequences are laid end to
-// end.  Group g of G (one group = 4 CTAs, one per 128-wide slice of the latent) streams
+// end.  Group g of G (one group = d_c / 128 CTAs, one per 128-wide slice of the latent) streams
 // the contiguous tile range [floor(g*T/G), floor((g+1)*T/G)), which may cover the end of
 // one sequence and the start of the next.  Each (group, sequence) pair it touches is one
 // "segment" and leaves one partial softmax state in workspace slot g + s; that map is

@@ -1,7 +1,7 @@
 """GPU parity: the CUDA path (through the C ABI) against the fp64 oracle on the same
 seeded inputs.  Small cases are compared element by element over every output; the five
 full-size workloads are compared on sampled (sequence, head) outputs in the launch
-configuration the benchmark uses (num_splits = 0: one split per 4 SMs)."""
+configuration the benchmark uses (num_splits = 0: one split per 4 SMs, one CTA per SM)."""
 import numpy as np
 import pytest
 import torch
