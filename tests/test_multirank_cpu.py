@@ -78,3 +78,29 @@ def test_reference_arm_prints_nothing_on_other_ranks():
         bench.run_reference(argparse.Namespace(steps=1, warmup=3, ref_seqs=1, ref_heads=1),
                             synth.WORKLOADS["small_mlra4_h16_t2k"], 2, 1)
     assert out.getvalue() == ""
+
+
+def test_reference_arm_for_a_branch_shard_reports_the_shard():
+    """--tp 4 on the reference arm times the oracle on rank 0's shard: one 128-wide branch
+    plus the rope key per token, strong scaling, and the shard's latent width in config."""
+    import argparse
+    import json
+
+    import bench
+    import synth
+    out = io.StringIO()
+    with contextlib.redirect_stdout(out):
+        bench.run_reference(argparse.Namespace(steps=1, warmup=3, ref_seqs=1, ref_heads=1, tp=4),
+                            synth.WORKLOADS["small_mlra4_h16_t2k"], 1, 0)
+    line = json.loads(out.getvalue())
+    assert line["impl"] == "reference" and line["scaling"] == "strong"
+    assert line["config"]["d_c"] == 128 and line["config"]["tp_shard"] == "1 of 4 branches per rank"
+    tokens = 2048
+    assert line["value"] == pytest.approx(tokens * (128 + 64) * 2 / (line["ms_per_step"] * 1e-3) / 1e12)
+    assert line["cpu_baseline"]["value"] == line["value"] and line["e2e"]["value"] == line["value"]
+
+
+def test_tensor_flops_per_token_of_a_shard():
+    import bench
+    assert bench.tensor_flops_per_token(4, 128) == 2176 * 128
+    assert bench.tensor_flops_per_token(1, 128, 128) == (2 * 192 + 2 * 128) * 128
