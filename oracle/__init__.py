@@ -10,8 +10,8 @@ identities and closed forms the pages fix, a library attention routine and hand-
 fixtures in ``tests/golden/``.  The pages print no worked numeric example of their
 own, so no pin compares against a number printed on the pages.
 """
-from .reference import (rope_rotate, mlra_decode_expanded, mlra_decode_absorbed, mla_decode,
+from .reference import (rope_rotate, mlra_decode_expanded, mlra_decode_absorbed, mla_decode, gla_decode,
                         mla_nope_key, mlra_nope_key_blocks, decode_batch)
 
-__all__ = ["rope_rotate", "mlra_decode_expanded", "mlra_decode_absorbed", "mla_decode",
+__all__ = ["rope_rotate", "mlra_decode_expanded", "mlra_decode_absorbed", "mla_decode", "gla_decode",
            "mla_nope_key", "mlra_nope_key_blocks", "decode_batch"]

@@ -223,6 +223,34 @@ def mla_decode(q, c_kv, k_rope, w_uk, w_uv, alpha_q: float = 1.0, alpha_kv: floa
     return np.stack(rows)
 
 
+def gla_decode(q, c_kv, k_rope, w_uk, w_uv, n_groups: int = 2, alpha_q: float = 1.0, alpha_kv: float = 1.0,
+               softmax_scale: float | None = None, rope_theta: float = 10000.0) -> np.ndarray:
+    """Grouped latent attention (GLA-n) decode for ONE sequence.
+
+    "Multi-Head Low-Rank Attention" (研究动机) describes GLA-2 as MLA's single latent head
+    split into two groups, so that each of 2 devices loads 2.5 d_h per token (its 256
+    latent columns and the shared rope key).  Reading (the page gives no more): the h
+    heads form n_groups contiguous groups of h / n_groups; head i of group g attends
+    with the MLA formula over latent columns [g*w, (g+1)*w), w = d_c / n_groups, and the
+    shared K_R; its W_UK[i], W_UV[i] are [w, d] (the group's rows only).  No branch sum.
+
+    q [h, d_nope + d_rope]; c_kv [L, d_c]; k_rope [L, d_rope]; w_uk [h, w, d_nope];
+    w_uv [h, w, d_v].  Returns float64 [h, d_v].
+    """
+    h, d_c = int(np.shape(q)[0]), int(np.shape(c_kv)[1])
+    if h % n_groups or d_c % n_groups:
+        raise ValueError(f"{h} heads / {d_c} latent columns do not split into {n_groups} groups")
+    w, per = d_c // n_groups, h // n_groups
+    c_kv = _f64(c_kv)
+    out = []
+    for g in range(n_groups):
+        heads = slice(g * per, (g + 1) * per)
+        out.append(mla_decode(_f64(q)[heads], c_kv[:, g * w:(g + 1) * w], k_rope, _f64(w_uk)[heads],
+                              _f64(w_uv)[heads], alpha_q=alpha_q, alpha_kv=alpha_kv,
+                              softmax_scale=softmax_scale, rope_theta=rope_theta))
+    return np.concatenate(out)
+
+
 def mla_nope_key(c_kv, w_uk_i) -> np.ndarray:
     """MLA's per-head no-position key C_KV W_UK^(i) over the whole latent, [L, d_nope]."""
     return _f64(c_kv) @ _f64(w_uk_i)

@@ -92,6 +92,43 @@ def test_mlra4_is_not_mla():
     assert _rel(mlra, mla) > 0.1
 
 
+@pytest.mark.parametrize("n_groups", [2, 4])
+def test_gla_is_mlra_with_the_other_groups_weights_zeroed(n_groups):
+    """GLA (head groups, each on its own latent group; "Multi-Head Low-Rank Attention",
+    研究动机) equals MLRA with branch = group, branch-sum scale 1, when each head's W_UK and
+    W_UV rows outside its group are zero: the other branches then have value 0.
+    Catches: heads assigned to the wrong group, the group's latent columns off by a block,
+    a dropped rope key."""
+    rng = np.random.default_rng(11)
+    h, L, d_c = 4, 23, 512
+    w = d_c // n_groups
+    q, c, kr, _, _ = _rand_case(rng, h=h, L=L, n_branch=n_groups)
+    wuk_g = rng.standard_normal((h, w, 128)) / math.sqrt(w)
+    wuv_g = rng.standard_normal((h, w, 128)) / math.sqrt(w)
+    wuk, wuv = np.zeros((h, d_c, 128)), np.zeros((h, d_c, 128))
+    for i in range(h):
+        g = i // (h // n_groups)
+        wuk[i, g * w:(g + 1) * w], wuv[i, g * w:(g + 1) * w] = wuk_g[i], wuv_g[i]
+    for kw in (dict(), dict(alpha_q=2.16, alpha_kv=3.74)):
+        gla = oracle.gla_decode(q, c, kr, wuk_g, wuv_g, n_groups, **kw)
+        mlra = oracle.mlra_decode_expanded(q, c, kr, wuk, wuv, n_groups, branch_scale=1.0, **kw)
+        assert _rel(gla, mlra) < 1e-12
+
+
+def test_gla_head_reads_only_its_group():
+    """A GLA-2 head's output does not change when the other group's latent columns do."""
+    rng = np.random.default_rng(12)
+    q, c, kr, _, _ = _rand_case(rng, h=4, L=17, n_branch=2, bf16=False)
+    wuk = rng.standard_normal((4, 256, 128)) / 16
+    wuv = rng.standard_normal((4, 256, 128)) / 16
+    base = oracle.gla_decode(q, c, kr, wuk, wuv, 2)
+    c2 = c.copy()
+    c2[:, 256:] += rng.standard_normal((17, 256))
+    moved = oracle.gla_decode(q, c2, kr, wuk, wuv, 2)
+    assert np.array_equal(moved[:2], base[:2])
+    assert _rel(moved[2:], base[2:]) > 1e-3
+
+
 # --- RoPE --------------------------------------------------------------------------------
 
 def test_rope_relative_position():
