@@ -43,9 +43,11 @@ import synth  # noqa: E402
 METRIC = "MLRA-4 decode µs/step & KV-cache read TB/s (fraction of ~8 TB/s HBM)"
 NOMINAL_HBM_GBS = 8000.0
 FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0}
-DECODE_SOURCES = ["head_rank_attention_b200/csrc/decode_split_sm100.cu", "head_rank_attention_b200/csrc/decode_sm100.cu",
-                  "head_rank_attention_b200/csrc/sm100.cuh", "head_rank_attention_b200/csrc/schedule.cuh",
-                  "head_rank_attention_b200/csrc/decode_sm100.h"]
+# The sources the 128-wide-branch decode kernel (the one whose ncu traffic is recorded) is
+# compiled from; a change to any of them invalidates the recorded traffic.
+DECODE_SOURCES = ["head_rank_attention_b200/csrc/decode_split_sm100.cu", "head_rank_attention_b200/csrc/sm100.cuh",
+                  "head_rank_attention_b200/csrc/schedule.cuh", "head_rank_attention_b200/csrc/decode_sm100.h",
+                  "head_rank_attention_b200/csrc/launch.h"]
 
 
 def tensor_flops_per_token(n_branch: int, heads: int, d_c: int = 512) -> int:

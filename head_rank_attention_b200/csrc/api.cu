@@ -65,11 +65,11 @@ hra_status validate(const hra_decode_params* p) {
   if (p->d_c == 512) {
     if (p->n_branch != 1 && p->n_branch != 2 && p->n_branch != 4)
       return fail(HRA_ERR_UNSUPPORTED, "n_branch=%d (supported with d_c=512: 1, 2, 4)", p->n_branch);
-  } else if (!((p->d_c == 128 || p->d_c == 256) && p->d_c == 128 * p->n_branch)) {
-    // a shard of 128-wide branches: d_c = 128 * (branches held)
+  } else if (!((p->d_c == 128 && p->n_branch == 1) || (p->d_c == 256 && (p->n_branch == 1 || p->n_branch == 2)))) {
+    // a shard of the latent: 128-wide branches (d_c = 128 * branches held) or one 256-wide branch
     return fail(HRA_ERR_UNSUPPORTED,
-                "d_c=%d with n_branch=%d (supported: d_c=512 with n_branch 1, 2, 4; or a shard of 128-wide "
-                "branches, d_c = 128 * n_branch = 128 or 256)",
+                "d_c=%d with n_branch=%d (supported: d_c=512 with n_branch 1, 2, 4; d_c=256 with n_branch 1, 2; "
+                "d_c=128 with n_branch 1)",
                 p->d_c, p->n_branch);
   }
   if (p->batch < 1 || p->batch > hra::kMaxBatch)

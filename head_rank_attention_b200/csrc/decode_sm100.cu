@@ -3,11 +3,13 @@
 // Step 2 of the decode in "Multi-Head Low-Rank Attention" (方法步骤详情): MQA-style
 // attention of the absorbed per-head queries over the shared key [C_KV | K_RoPE] and
 // value C_KV, one independent softmax per (head, branch) (核心方法:
-// O = sum_b Softmax(Q K_b^T) V_b; MLA is the single-branch case).  This kernel serves MLA
-// (NB = 1) and MLRA-2 (NB = 2); MLRA-4 runs decode_split_sm100.cu.
+// O = sum_b Softmax(Q K_b^T) V_b; MLA is the single-branch case).  This kernel serves
+// branches 512 wide (NB = 1: MLA) and 256 wide (NB = 2: MLRA-2, or a call holding one
+// 256-wide latent group: a rank of MLRA-2 split by branch, or of GLA-2); 128-wide branches
+// run decode_split_sm100.cu.
 //
 // Work decomposition (one CTA per SM):
-//   blockIdx.x = slice c in 0..3: the CTA owns output latent columns [128c, 128c+128),
+//   blockIdx.x = slice c in 0..d_c/128-1: the CTA owns output latent columns [128c, 128c+128),
 //                which belong to branch b = c / (W/128) of width W = 512/NB;
 //   blockIdx.y = group g: a contiguous range of cache tiles (see schedule.cuh).
 // A CTA streams, for every tile of NT tokens, the branch's W latent columns plus the 64
@@ -349,12 +351,12 @@ decode_kernel(const __grid_constant__ CUtensorMap map_ckv, const __grid_constant
       // the two halves store alternate 64-column chunks.
       {
         const uint4* qsrc = reinterpret_cast<const uint4*>(
-            a.q_tilde + (static_cast<long long>(s) * a.heads + min(row, a.heads - 1)) * 576);
+            a.q_tilde + (static_cast<long long>(s) * a.heads + min(row, a.heads - 1)) * (a.d_c + 64));
         const bool live = row < a.heads;
         uint32_t w[32];
 #pragma unroll 1
         for (int c = half; c < C::QK_DIMS / 64; c += 2) {
-          const int col0 = (c < C::QK_DIMS / 64 - 1) ? branch * C::W + 64 * c : 512;  // fp16 column
+          const int col0 = (c < C::QK_DIMS / 64 - 1) ? branch * C::W + 64 * c : a.d_c;  // fp16 column
 #pragma unroll
           for (int u = 0; u < 8; ++u) {
             const uint4 v = live ? __ldg(qsrc + (col0 >> 3) + u) : make_uint4(0u, 0u, 0u, 0u);
@@ -444,7 +446,8 @@ decode_kernel(const __grid_constant__ CUtensorMap map_ckv, const __grid_constant
       if (!warp_wait(pv_done, (it - 1) & 1, limit, abort_flag, status, 32)) { ok = false; break; }
       tc_fence_after();
       const long long slot = static_cast<long long>(g) + s;
-      float4* dst = reinterpret_cast<float4*>(a.o_part + ((slot * 4 + slice) * 128 + row) * 128 + 64 * half);
+      float4* dst =
+          reinterpret_cast<float4*>(a.o_part + ((slot * gridDim.x + slice) * 128 + row) * 128 + 64 * half);
 #pragma unroll 1
       for (int k = 0; k < 2; ++k) {
         uint32_t o[32];
@@ -463,7 +466,7 @@ decode_kernel(const __grid_constant__ CUtensorMap map_ckv, const __grid_constant
       if (!warp_wait(lsum_bar, seg & 1, limit, abort_flag, status, 34)) { ok = false; break; }
       ++seg;
       if (half == 0 && row < a.heads)
-        a.ml_part[(slot * 4 + slice) * 128 + row] = make_float2(m_ref, l + red_l[128 + row]);
+        a.ml_part[(slot * gridDim.x + slice) * 128 + row] = make_float2(m_ref, l + red_l[128 + row]);
       tc_fence_before();
     }
   }
@@ -483,7 +486,8 @@ cudaError_t launch_decode(const CUtensorMap& map_ckv, const CUtensorMap& map_kro
   auto kern = decode_kernel<NB, NT, STAGES>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
   if (e != cudaSuccess) return e;
-  return launch_kernel(kern, dim3(4, groups), dim3(C::THREADS), C::SMEM_BYTES, stream, pdl, map_ckv, map_krope, a);
+  return launch_kernel(kern, dim3(a.d_c / 128, groups), dim3(C::THREADS), C::SMEM_BYTES, stream, pdl, map_ckv,
+                       map_krope, a);
 }
 
 }  // namespace
@@ -494,12 +498,11 @@ int decode_tile_tokens(int branch_width) {
 
 cudaError_t launch_decode_kernel(int n_branch, const CUtensorMap& map_ckv, const CUtensorMap& map_krope,
                                  const DecodeArgs& a, int groups, cudaStream_t stream, bool pdl) {
-  if (n_branch < 1 || a.d_c % n_branch != 0) return cudaErrorInvalidValue;
-  if (a.d_c / n_branch == 128) return launch_decode_split_kernel(map_ckv, map_krope, a, groups, stream, pdl);
-  if (a.d_c != 512) return cudaErrorInvalidValue;  // this kernel assumes the whole 512-wide latent
-  switch (n_branch) {
-    case 2: return launch_decode<2, 64, 5>(map_ckv, map_krope, a, groups, stream, pdl);
-    case 1: return launch_decode<1, 32, 5>(map_ckv, map_krope, a, groups, stream, pdl);
+  if (n_branch < 1 || a.d_c % n_branch != 0 || a.d_c % 128 != 0 || a.d_c > 512) return cudaErrorInvalidValue;
+  switch (a.d_c / n_branch) {  // branch width
+    case 128: return launch_decode_split_kernel(map_ckv, map_krope, a, groups, stream, pdl);
+    case 256: return launch_decode<2, 64, 5>(map_ckv, map_krope, a, groups, stream, pdl);
+    case 512: return launch_decode<1, 32, 5>(map_ckv, map_krope, a, groups, stream, pdl);
     default: return cudaErrorInvalidValue;
   }
 }

@@ -62,7 +62,7 @@ cudaError_t launch_decode_split_kernel(const CUtensorMap& map_ckv, const CUtenso
 
 // Launch the decode kernel on grid (d_c / 128 slices, `groups` KV splits); pdl:
 // programmatic dependent launch (launch.h).  Branches 128 wide run the split kernel, 256
-// and 512 wide (d_c = 512 only) the converting kernel.
+// and 512 wide the converting kernel.
 cudaError_t launch_decode_kernel(int n_branch, const CUtensorMap& map_ckv, const CUtensorMap& map_krope,
                                  const DecodeArgs& a, int groups, cudaStream_t stream, bool pdl);
 

@@ -18,6 +18,10 @@
  * d_c = 128 * n_branch in {128, 256} computes the branches it holds, and its out is that
  * shard's part of the branch sum; summing out over the shards (an all-reduce across the
  * devices) gives the MLRA-4 output.  Pass the full model's branch_scale (1/2 for MLRA-4).
+ * A call with d_c = 256 and n_branch = 1 attends over one 256-wide latent: a rank of MLRA-2
+ * split by branch (branch_scale 1/sqrt(2), outs summed), or a rank of GLA-2 (研究动机: MLA's
+ * latent split into two groups; the rank's heads only, branch_scale 1, outs concatenated
+ * over heads).
  * The softmax scale of every branch is 1/sqrt(d_nope + d_rope) by default
  * ("vllbc02MLA", DeepseekV2Attention.__init__: scaling = qk_head_dim ** -0.5).
  *
@@ -28,12 +32,12 @@
  * Bounded device waits that expire write a status word in the workspace, read back
  * by hra_check_device_status().
  * Numerics: bf16 inputs, fp32 accumulation; softmax, combine and up-projection in fp32.
- * 128-wide branches (n_branch = 4, and branch shards): the tensor cores read the latent
+ * 128-wide branches (d_c / n_branch = 128): the tensor cores read the latent
  * part of the cache as stored, against
  * the absorbed query carried as two bf16 terms (hi + lo, ~16 significant bits); the rope
  * part (query and K_RoPE tile) is scored in fp16, so |K_RoPE values| must stay below 65504.
- * n_branch = 1, 2: the cache tile is converted to fp16 in shared memory and the query is
- * fp16, so |cache values| must stay below 65504.
+ * 256- and 512-wide branches: the cache tile is converted to fp16 in shared memory and the
+ * query is fp16, so |cache values| must stay below 65504.
  * Stream order: the kernels of a call are chained with programmatic dependent launch, so
  * a call may begin (set-up, loads of its inputs) while the previous call on the stream
  * drains; it touches the workspace only once that call has completed.
@@ -68,7 +72,7 @@ typedef enum { HRA_BF16 = 0, HRA_F32 = 1 } hra_dtype;
 /*
  * Parameters of one decode step.  All pointers are device pointers, 16-byte aligned.
  * Supported set: d_rope = 64, d_nope = 128, d_v = 128; d_c = 512 with n_branch in {1,2,4},
- * or a branch shard d_c = 128 * n_branch in {128, 256}; 1 <= num_heads <= 128,
+ * d_c = 256 with n_branch in {1,2}, d_c = 128 with n_branch = 1; 1 <= num_heads <= 128,
  * 1 <= batch <= 1024.
  */
 typedef struct {

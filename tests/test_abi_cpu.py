@@ -66,7 +66,8 @@ def _fake_params(**over):
     return p
 
 
-@pytest.mark.parametrize("d_c,n_branch,splits", [(512, 4, 37), (512, 1, 37), (256, 2, 74), (128, 1, 148)])
+@pytest.mark.parametrize("d_c,n_branch,splits", [(512, 4, 37), (512, 1, 37), (256, 2, 74), (256, 1, 74),
+                                                   (128, 1, 148)])
 def test_workspace_size_formula(d_c, n_branch, splits):
     p = _fake_params(d_c=d_c, n_branch=n_branch, num_splits=splits, ckv_stride=d_c + 64, krope_stride=d_c + 64)
     n = hra.workspace_size(p)
@@ -85,7 +86,6 @@ def test_workspace_size_formula(d_c, n_branch, splits):
     (dict(ckv=0x20008), B.HRA_ERR_INVALID_ARG),          # misaligned
     (dict(n_branch=3), B.HRA_ERR_UNSUPPORTED),
     (dict(d_c=256), B.HRA_ERR_UNSUPPORTED),
-    (dict(d_c=256, n_branch=1, ckv_stride=320), B.HRA_ERR_UNSUPPORTED),   # a 256-wide branch shard
     (dict(d_c=128, n_branch=2, ckv_stride=192), B.HRA_ERR_UNSUPPORTED),   # 64-wide branches
     (dict(d_c=384, n_branch=3, ckv_stride=448), B.HRA_ERR_UNSUPPORTED),
     (dict(d_c=128, n_branch=1, ckv_stride=120), B.HRA_ERR_INVALID_ARG),   # stride below d_c

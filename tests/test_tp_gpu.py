@@ -140,3 +140,77 @@ def test_shard_paged_equals_contiguous_bitwise():
         wl = _wl("layout", lens, page_size=page_size)
         outs.append(_run_shard(synth.to_device(synth.make_inputs(wl)), wl, 2, 4, 0))
     assert torch.equal(outs[0], outs[1])
+
+
+# --- one 256-wide latent per call: MLRA-2 split by branch, and GLA-2 ranks -------------------
+
+def _wl2(name, lengths, heads=128, page_size=0, **kw):
+    return synth.Workload(name, 2, len(lengths), heads, max(lengths), page_size=page_size,
+                          lengths=tuple(lengths), **kw)
+
+
+CASES_256 = [
+    _wl2("tails", (1, 31, 32, 33, 63, 64, 65, 1000)),
+    _wl2("paged32", (5, 64, 65, 700), page_size=32),
+    _wl2("stress", (3000, 17), alpha_q=synth.A_Q_V3, alpha_kv=synth.A_KV_V3),
+]
+
+
+def _call(q, local, w_uk, w_uv, dev, wl, n_branch, branch_scale):
+    d = local.shape[1] - synth.D_ROPE
+    out = torch.empty(q.shape[0], q.shape[1], synth.D_V, dtype=torch.float32, device="cuda")
+    p = hra.make_params(q, local[:, :d], local[:, d:], dev.seq_lens, w_uk, w_uv, out, n_branch=n_branch,
+                        alpha_q=wl.alpha_q, alpha_kv=wl.alpha_kv, branch_scale=branch_scale,
+                        softmax_scale=wl.softmax_scale, rope_theta=wl.rope_theta, block_table=dev.block_table,
+                        page_size=wl.page_size, seq_stride=dev.seq_stride)
+    ws = hra.alloc_workspace(p)
+    ws.fill_(0xFF)
+    hra.mlra_decode(p)
+    hra.check_device_status(p)
+    return out
+
+
+@pytest.mark.parametrize("wl", CASES_256, ids=lambda w: w.name)
+def test_mlra2_branch_shards_sum_to_mlra2(wl):
+    """2-way tensor parallelism of MLRA-2: each rank holds one 256-wide branch (d_c = 256,
+    n_branch = 1, branch_scale 1/sqrt(2)); the ranks' outputs sum to MLRA-2's."""
+    inp = synth.make_inputs(wl)
+    dev = synth.to_device(inp)
+    total = torch.zeros(wl.batch, wl.heads, synth.D_V, dtype=torch.float32, device="cuda")
+    for r in range(2):
+        local = tp.shard_cache(dev.cache, r, 2, n_branch=2)
+        w_uk, w_uv = tp.shard_weights(dev.w_uk, dev.w_uv, r, 2, n_branch=2)
+        out = _call(dev.q, local, w_uk, w_uv, dev, wl, 1, wl.sigma_o)
+        h_uk, h_uv = tp.shard_weights(inp.w_uk, inp.w_uv, r, 2, n_branch=2)
+        ref = np.stack([oracle.mlra_decode_absorbed(
+            inp.q[s], *(lambda x: (x[:, :256], x[:, 256:]))(tp.shard_cache(synth.logical_rows(inp, wl, s), r, 2,
+                                                                           n_branch=2)),
+            h_uk, h_uv, 1, alpha_q=wl.alpha_q, alpha_kv=wl.alpha_kv, branch_scale=wl.sigma_o,
+            softmax_scale=wl.softmax_scale, rope_theta=wl.rope_theta) for s in range(wl.batch)])
+        assert_parity(out.cpu().numpy(), ref, f"{wl.name} MLRA-2 shard {r}/2")
+        total += out
+    assert_parity(total.cpu().numpy(), oracle.decode_batch(inp, wl, form="absorbed"), f"{wl.name} MLRA-2 sum")
+
+
+@pytest.mark.parametrize("wl", CASES_256[:2], ids=lambda w: w.name)
+def test_gla2_ranks_match_the_oracle(wl):
+    """GLA-2 (研究动机: MLA's latent split into two groups): rank g holds latent group g and
+    the heads of group g; its call is MLA over a 256-wide latent.  Head i's weights are the
+    group's rows of the seeded [h, 512, 128] weights."""
+    inp = synth.make_inputs(wl)
+    dev = synth.to_device(inp)
+    h, per = wl.heads, wl.heads // 2
+    w_uk = torch.stack([inp.w_uk[i, (i // per) * 256:(i // per + 1) * 256] for i in range(h)])
+    w_uv = torch.stack([inp.w_uv[i, (i // per) * 256:(i // per + 1) * 256] for i in range(h)])
+    outs = []
+    for g in range(2):
+        heads = slice(g * per, (g + 1) * per)
+        local = tp.shard_cache(dev.cache, g, 2, n_branch=2)
+        outs.append(_call(dev.q[:, heads].contiguous(), local, w_uk[heads].cuda().contiguous(),
+                          w_uv[heads].cuda().contiguous(), dev, wl, 1, 1.0))
+    got = torch.cat(outs, dim=1).cpu().numpy()
+    ref = np.stack([oracle.gla_decode(inp.q[s], (r := synth.logical_rows(inp, wl, s))[:, :512], r[:, 512:],
+                                      w_uk, w_uv, 2, alpha_q=wl.alpha_q, alpha_kv=wl.alpha_kv,
+                                      softmax_scale=wl.softmax_scale, rope_theta=wl.rope_theta)
+                    for s in range(wl.batch)])
+    assert_parity(got, ref, f"{wl.name} GLA-2")
