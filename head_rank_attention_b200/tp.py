@@ -11,6 +11,11 @@ and the full model's branch_scale; its output is that shard's part of the branch
 and one all-reduce (sum) over the tensor-parallel group gives the model's output.  This
 module lays the cache and weights out per shard and does that all-reduce; the decode
 itself runs in libhra.so.
+
+The same layout serves MLRA-2 split by branch over 2 ranks (n_branch=2: one 256-wide
+branch per rank, a d_c = 256, n_branch = 1 call) and the latent side of a GLA-2 rank
+(研究动机: MLA's latent split into two groups; the rank also holds only its group's heads,
+and the ranks' outputs are concatenated over heads instead of summed).
 """
 from __future__ import annotations
 
