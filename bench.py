@@ -12,10 +12,10 @@ Multi-GPU (torchrun, one rank per GPU): every rank decodes its own replica batch
 path has no exchange step); value = all ranks' KV bytes / max-over-ranks step time.
 One JSON line is printed by rank 0.
 
---tp W (W = 2 or 4, MLRA-4 workloads): tensor parallelism by branch.  Rank r holds its
-W-th of the branches (cache columns + K_RoPE, W_UK / W_UV rows) and a step is its shard's
-decode followed by an NCCL all-reduce of out; run it with --gpus W.  With one GPU, the
-rank-0 shard's step is timed alone (no all-reduce).
+--tp W (W = 2 or 4 for MLRA-4, 2 for MLRA-2): tensor parallelism by branch.  Rank r holds
+its W-th of the branches (cache columns + K_RoPE, W_UK / W_UV rows) and a step is its
+shard's decode followed by an NCCL all-reduce of out; run it with --gpus W.  With one GPU,
+the rank-0 shard's step is timed alone (no all-reduce).
 """
 from __future__ import annotations
 
@@ -167,8 +167,8 @@ def time_oracle_sample(wl: synth.Workload, n_seqs: int, n_heads: int, tp_world: 
     rows = {s: synth.seq_rows(wl, s) for s in seqs}  # generation is not timed
     d_c, n_branch = synth.D_C, wl.n_branch
     if tp_world:
-        rows = {s: tp.shard_cache(r, 0, tp_world) for s, r in rows.items()}
-        w_uk, w_uv = tp.shard_weights(w_uk, w_uv, 0, tp_world)
+        rows = {s: tp.shard_cache(r, 0, tp_world, n_branch) for s, r in rows.items()}
+        w_uk, w_uv = tp.shard_weights(w_uk, w_uv, 0, tp_world, n_branch)
         d_c, n_branch = synth.D_C // tp_world, wl.n_branch // tp_world
     t0 = time.perf_counter()
     for s in seqs:
@@ -188,7 +188,7 @@ def workload_config(wl: synth.Workload, lens, tp_world: int = 0) -> dict:
             "seq_len_min": wl.seq_len_min, "total_tokens": int(np.asarray(lens, dtype=np.int64).sum()),
             "layout": f"paged({wl.page_size})" if wl.page_size else "contiguous",
             "d_c": 512 // tp_world if tp_world else 512, "d_rope": 64,
-            **({"tp_shard": f"{4 // tp_world} of 4 branches per rank"} if tp_world else {}), "alpha_q": wl.alpha_q, "alpha_kv": wl.alpha_kv, "branch_scale": wl.sigma_o,
+            **({"tp_shard": f"{wl.n_branch // tp_world} of {wl.n_branch} branches per rank"} if tp_world else {}), "alpha_q": wl.alpha_q, "alpha_kv": wl.alpha_kv, "branch_scale": wl.sigma_o,
             "l2": "inputs larger than L2 (KV cache per step >> 126 MB); no flush"}
 
 
@@ -260,10 +260,10 @@ def run_native(args, wl, world, rank, local):
     host_cache, host_wuk, host_wuv = inp.cache, inp.w_uk, inp.w_uv
     if tpw:  # this rank's branch shard (rank 0's when one GPU stands alone)
         shard = rank if world == tpw else 0
-        cache = hra.tp.shard_cache(dev.cache, shard, tpw)
-        w_uk, w_uv = hra.tp.shard_weights(dev.w_uk, dev.w_uv, shard, tpw)
-        host_cache = hra.tp.shard_cache(inp.cache, shard, tpw)
-        host_wuk, host_wuv = hra.tp.shard_weights(inp.w_uk, inp.w_uv, shard, tpw)
+        cache = hra.tp.shard_cache(dev.cache, shard, tpw, wl.n_branch)
+        w_uk, w_uv = hra.tp.shard_weights(dev.w_uk, dev.w_uv, shard, tpw, wl.n_branch)
+        host_cache = hra.tp.shard_cache(inp.cache, shard, tpw, wl.n_branch)
+        host_wuk, host_wuv = hra.tp.shard_weights(inp.w_uk, inp.w_uv, shard, tpw, wl.n_branch)
         dev.cache = dev.w_uk = dev.w_uv = None
         torch.cuda.empty_cache()
         d_c, n_branch = synth.D_C // tpw, wl.n_branch // tpw
@@ -483,8 +483,8 @@ def main():
         ap.error("--warmup must be >= 3")
     world, rank, local = dist_setup()
     wl = synth.WORKLOADS[args.workload]
-    if args.tp and wl.n_branch != 4:
-        ap.error("--tp needs an MLRA-4 workload (128-wide branches)")
+    if args.tp and (wl.n_branch == 1 or wl.n_branch % args.tp != 0):
+        ap.error(f"--tp {args.tp} needs whole branches per rank (MLRA-4: 2 or 4; MLRA-2: 2)")
     if args.tp and world not in (1, args.tp):
         ap.error(f"--tp {args.tp} runs on {args.tp} ranks (or one GPU for a single shard), not {world}")
     if args.impl == "reference":
