@@ -50,6 +50,7 @@ class HraDecodeParams(ctypes.Structure):
         ("workspace", ctypes.c_void_p), ("workspace_bytes", ctypes.c_size_t),
         ("num_splits", ctypes.c_int), ("wait_limit", ctypes.c_int),
         ("stage_events", ctypes.c_void_p),
+        ("out_accumulate", ctypes.c_int), ("n_out_peers", ctypes.c_int), ("out_peers", ctypes.c_void_p),
     ]
 
 
@@ -108,11 +109,14 @@ def make_params(q, ckv, krope, seq_lens, w_uk, w_uv, out, workspace=None, *, n_b
                 alpha_q: float = 1.0, alpha_kv: float = 1.0, branch_scale: Optional[float] = None,
                 softmax_scale: float = 0.0, rope_theta: float = 10000.0, block_table=None,
                 page_size: int = 0, seq_stride: int = 0, cache_rows: Optional[int] = None,
-                num_splits: int = 0, wait_limit: int = 0) -> HraDecodeParams:
+                num_splits: int = 0, wait_limit: int = 0, out_accumulate: bool = False,
+                out_peers=None) -> HraDecodeParams:
     """Fill hra_decode_params from torch tensors (shapes/dtypes as documented in hra.h).
 
     ckv / krope are 2-D row views of the cache (e.g. cache[:, :512], cache[:, 512:]);
-    their row strides become ckv_stride / krope_stride.
+    their row strides become ckv_stride / krope_stride.  out_peers: device addresses (ints)
+    or tensors of other ranks' out buffers for out_accumulate (the array is kept alive on
+    the returned object).
     """
     import torch
     p = HraDecodeParams()
@@ -136,6 +140,11 @@ def make_params(q, ckv, krope, seq_lens, w_uk, w_uv, out, workspace=None, *, n_b
     p.workspace = _ptr(workspace)
     p.workspace_bytes = 0 if workspace is None else int(workspace.numel() * workspace.element_size())
     p.num_splits, p.wait_limit = int(num_splits), int(wait_limit)
+    p.out_accumulate = int(bool(out_accumulate))
+    peers = [x if isinstance(x, int) else _ptr(x) for x in (out_peers or [])]
+    p._out_peers = (ctypes.c_void_p * max(1, len(peers)))(*peers)
+    p.out_peers = ctypes.cast(p._out_peers, ctypes.c_void_p).value if peers else None
+    p.n_out_peers = len(peers)
     return p
 
 

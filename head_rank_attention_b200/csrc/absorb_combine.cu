@@ -470,7 +470,18 @@ upproj_tc_kernel(const __grid_constant__ CUtensorMap map_wuv, const __grid_const
       tmem_ld_wait();
       if (s < a.batch) {
         const long long o = (static_cast<long long>(s) * a.heads + i) * 128 + d0;
-        if (a.out_f32) {
+        if (a.out_f32 && a.accumulate) {
+          // this call's part of a sum over calls (tensor-parallel ranks): add it into this
+          // rank's out and into every peer's, over NVLink for peer memory
+#pragma unroll
+          for (int q = 0; q < 8; ++q) {
+            const float4 x =
+                make_float4(scale * __uint_as_float(v[4 * q]), scale * __uint_as_float(v[4 * q + 1]),
+                            scale * __uint_as_float(v[4 * q + 2]), scale * __uint_as_float(v[4 * q + 3]));
+            atomicAdd(reinterpret_cast<float4*>(a.out_f32 + o + 4 * q), x);
+            for (int k = 0; k < a.n_peers; ++k) atomicAdd(reinterpret_cast<float4*>(a.peers[k] + o + 4 * q), x);
+          }
+        } else if (a.out_f32) {
 #pragma unroll
           for (int q = 0; q < 8; ++q)
             *reinterpret_cast<float4*>(a.out_f32 + o + 4 * q) =

@@ -22,6 +22,8 @@ struct AbsorbArgs {
   float alpha_q, alpha_kv, rope_theta;
 };
 
+constexpr int kMaxOutPeers = 7;  // other ranks' out buffers the up-projection can add into
+
 struct CombineArgs {
   const float* o_part;        // [slots, d_c / 128, 128, 128]
   const float2* ml_part;      // [slots, d_c / 128, 128]
@@ -30,6 +32,9 @@ struct CombineArgs {
   int* status;                // device status word (expired waits)
   float* out_f32;             // [B, h, 128] or nullptr
   __nv_bfloat16* out_bf16;    // [B, h, 128] or nullptr
+  int accumulate;             // 1: add into out_f32 and every peers[k] (fp32 atomics) instead of storing
+  int n_peers;
+  float* peers[kMaxOutPeers]; // other ranks' out buffers (peer memory), [B, h, 128] fp32
   int batch, heads, groups;
   int d_c;                    // latent width (as in AbsorbArgs)
   float alpha_kv, branch_scale;

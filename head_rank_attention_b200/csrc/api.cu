@@ -101,6 +101,19 @@ hra_status validate(const hra_decode_params* p) {
   if (p->out_dtype != HRA_BF16 && p->out_dtype != HRA_F32)
     return fail(HRA_ERR_INVALID_ARG, "out_dtype=%d", (int)p->out_dtype);
   if (p->num_splits < 0) return fail(HRA_ERR_INVALID_ARG, "num_splits=%d must be >= 0", p->num_splits);
+  if (p->out_accumulate != 0 && p->out_accumulate != 1)
+    return fail(HRA_ERR_INVALID_ARG, "out_accumulate=%d must be 0 or 1", p->out_accumulate);
+  if (p->out_accumulate && p->out_dtype != HRA_F32)
+    return fail(HRA_ERR_INVALID_ARG, "out_accumulate needs out_dtype = HRA_F32");
+  if (p->n_out_peers < 0 || p->n_out_peers > hra::kMaxOutPeers)
+    return fail(HRA_ERR_UNSUPPORTED, "n_out_peers=%d (supported: 0..%d)", p->n_out_peers, hra::kMaxOutPeers);
+  if (p->n_out_peers > 0) {
+    if (!p->out_accumulate) return fail(HRA_ERR_INVALID_ARG, "out_peers need out_accumulate = 1");
+    if (p->out_peers == nullptr) return fail(HRA_ERR_INVALID_ARG, "out_peers is NULL");
+    for (int k = 0; k < p->n_out_peers; ++k)
+      if (p->out_peers[k] == nullptr || !aligned16(p->out_peers[k]))
+        return fail(HRA_ERR_INVALID_ARG, "out_peers[%d] is NULL or not 16-byte aligned", k);
+  }
   if (p->wait_limit < 0) return fail(HRA_ERR_INVALID_ARG, "wait_limit=%d must be >= 0", p->wait_limit);
   if (!std::isfinite(p->alpha_q) || !std::isfinite(p->alpha_kv) || !std::isfinite(p->branch_scale) ||
       !std::isfinite(p->softmax_scale) || !(p->rope_theta > 0.f) || !std::isfinite(p->rope_theta))
@@ -252,6 +265,9 @@ hra_status run_decode(const hra_decode_params* p, cudaStream_t stream) {
   cb.status = status;
   cb.out_f32 = p->out_dtype == HRA_F32 ? static_cast<float*>(p->out) : nullptr;
   cb.out_bf16 = p->out_dtype == HRA_BF16 ? static_cast<__nv_bfloat16*>(p->out) : nullptr;
+  cb.accumulate = p->out_accumulate;
+  cb.n_peers = p->n_out_peers;
+  for (int k = 0; k < p->n_out_peers; ++k) cb.peers[k] = static_cast<float*>(p->out_peers[k]);
   cb.batch = p->batch;
   cb.heads = p->num_heads;
   cb.groups = plan.groups;

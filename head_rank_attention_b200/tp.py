@@ -23,7 +23,7 @@ from typing import Optional, Tuple
 
 import torch
 
-__all__ = ["shard_columns", "shard_cache", "shard_weights", "all_reduce_out"]
+__all__ = ["shard_columns", "shard_cache", "shard_weights", "all_reduce_out", "peer_ranks", "PeerOut"]
 
 
 def shard_columns(d_c: int, n_branch: int, rank: int, world: int) -> Tuple[int, int]:
@@ -50,6 +50,50 @@ def shard_weights(w_uk: torch.Tensor, w_uv: torch.Tensor, rank: int, world: int,
     """Rank `rank`'s rows of W_UK and W_UV ([h, d_c, 128] each): [h, c1 - c0, 128]."""
     c0, c1 = shard_columns(int(w_uk.shape[1]), n_branch, rank, world)
     return w_uk[:, c0:c1].contiguous(), w_uv[:, c0:c1].contiguous()
+
+
+def peer_ranks(rank: int, world: int) -> list:
+    """The ranks whose out buffers a rank's up-projection adds into besides its own, in
+    rank order (the order of hra_decode_params.out_peers)."""
+    if not 0 <= rank < world:
+        raise ValueError(f"rank {rank} outside [0, {world})")
+    return [r for r in range(world) if r != rank]
+
+
+class PeerOut:
+    """Out buffers for the fused up-projection + all-reduce of a branch-sharded decode.
+
+    Every rank allocates its fp32 out [B, h, d_v] in symmetric memory (peer-mapped over
+    NVLink) and learns the addresses of the other ranks' buffers.  A step is then
+
+        po.begin()                    # zero this rank's out; barrier: every out is zeroed
+        p = make_params(..., out=po.out, out_accumulate=True, out_peers=po.peers)
+        mlra_decode(p)                # adds this shard's part into every rank's out
+        po.end()                      # barrier: every rank's additions have landed
+
+    after which po.out holds the sum over the shards on every rank.  The barriers are
+    torch's symmetric-memory device barriers on the current stream (bounded by
+    timeout_ms), so no host synchronisation sits in the step.
+    """
+
+    def __init__(self, shape, group=None, device=None, timeout_ms: int = 10000):
+        import torch.distributed as dist
+        import torch.distributed._symmetric_memory as symm_mem
+        group = dist.group.WORLD if group is None else group
+        self.out = symm_mem.empty(*shape, dtype=torch.float32, device=device)
+        self.handle = symm_mem.rendezvous(self.out, group)
+        self.rank, self.world = int(self.handle.rank), int(self.handle.world_size)
+        ptrs = list(self.handle.buffer_ptrs)
+        self.peers = [int(ptrs[r]) for r in peer_ranks(self.rank, self.world)]
+        self.timeout_ms = int(timeout_ms)
+
+    def begin(self) -> None:
+        self.out.zero_()
+        self.handle.barrier(channel=0, timeout_ms=self.timeout_ms)
+
+    def end(self) -> torch.Tensor:
+        self.handle.barrier(channel=1, timeout_ms=self.timeout_ms)
+        return self.out
 
 
 def all_reduce_out(out: torch.Tensor, group: Optional[object] = None) -> torch.Tensor:

@@ -121,6 +121,19 @@ typedef struct {
   void* const* stage_events; /* optional, NULL = none: 4 caller-owned cudaEvent_t recorded on
                                 `stream` before absorption, before the split-KV decode, before
                                 the combine/up-projection and after it (per-stage timing)    */
+
+  /* Tensor-parallel output, fused with the up-projection (optional; 0 = off).
+     out_accumulate = 1: instead of storing out, the up-projection ADDS its result (fp32
+     atomics; out_dtype must be HRA_F32) into out and into each out_peers[k].  With
+     out_peers = the other ranks' out buffers mapped into this process (peer memory over
+     NVLink: symmetric memory or IPC), every rank of a branch-sharded call writes its
+     shard's part of the branch sum into every rank's out, so the sum over shards needs no
+     separate all-reduce.  The caller zeroes the buffers and orders the ranks: every out is
+     zeroed before any rank's call starts, and read only after every rank's call completed.
+     The order of the additions varies, so the sum is not bitwise reproducible.          */
+  int out_accumulate;   /* 0 or 1                                                        */
+  int n_out_peers;      /* 0..7 entries in out_peers (requires out_accumulate = 1)        */
+  void* const* out_peers; /* host array of device pointers to [B, h, d_v] fp32, 16-B aligned */
 } hra_decode_params;
 
 /* Bytes of workspace one call with these parameters needs (0 on invalid parameters).

@@ -107,6 +107,41 @@ def test_validation_rejects_before_launch(over, status):
     assert hra.last_error() != ""
 
 
+_GOOD_PEERS = (ctypes.c_void_p * 2)(0x90000, 0xA0000)
+_BAD_PEERS = (ctypes.c_void_p * 2)(0x90000, 0xA0008)
+
+
+@pytest.mark.parametrize("over,status", [
+    (dict(out_accumulate=2), B.HRA_ERR_INVALID_ARG),
+    (dict(out_accumulate=1, out_dtype=B.HRA_BF16), B.HRA_ERR_INVALID_ARG),
+    (dict(out_accumulate=1, n_out_peers=8, out_peers=ctypes.addressof(_GOOD_PEERS)), B.HRA_ERR_UNSUPPORTED),
+    (dict(n_out_peers=2, out_peers=ctypes.addressof(_GOOD_PEERS)), B.HRA_ERR_INVALID_ARG),  # no accumulate
+    (dict(out_accumulate=1, n_out_peers=2, out_peers=None), B.HRA_ERR_INVALID_ARG),
+    (dict(out_accumulate=1, n_out_peers=2, out_peers=ctypes.addressof(_BAD_PEERS)), B.HRA_ERR_INVALID_ARG),
+    (dict(out_accumulate=1, n_out_peers=2, out_peers=ctypes.addressof(_GOOD_PEERS)), B.HRA_ERR_WORKSPACE),
+])
+def test_fused_output_fields_are_validated(over, status):
+    """The fused tensor-parallel output (out_accumulate, out_peers) is checked before any
+    launch; a well-formed one passes validation (and stops at the missing workspace)."""
+    p = _fake_params(**over)
+    rc = hra.load_library().mlra_decode(ctypes.byref(p), None)
+    assert rc == status, hra.last_error()
+
+
+def test_make_params_fills_the_peer_array():
+    import torch
+    q = torch.zeros(1, 4, 192, dtype=torch.bfloat16)
+    cache = torch.zeros(64, 576, dtype=torch.bfloat16)
+    w = torch.zeros(4, 512, 128, dtype=torch.bfloat16)
+    out = torch.zeros(1, 4, 128)
+    p = hra.make_params(q, cache[:, :512], cache[:, 512:], torch.zeros(1, dtype=torch.int32), w, w, out,
+                        n_branch=4, out_accumulate=True, out_peers=[0x1000, 0x2000])
+    assert p.out_accumulate == 1 and p.n_out_peers == 2
+    assert list((ctypes.c_void_p * 2).from_address(p.out_peers)) == [0x1000, 0x2000]
+    p0 = hra.make_params(q, cache[:, :512], cache[:, 512:], torch.zeros(1, dtype=torch.int32), w, w, out, n_branch=4)
+    assert p0.out_accumulate == 0 and p0.n_out_peers == 0 and not p0.out_peers
+
+
 def test_mla_decode_requires_one_branch():
     p = _fake_params(n_branch=4)
     with pytest.raises(hra.HraError) as e:

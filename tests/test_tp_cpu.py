@@ -53,6 +53,14 @@ def test_shard_columns():
             tp.shard_columns(*bad)
 
 
+def test_peer_ranks():
+    assert tp.peer_ranks(0, 1) == []
+    assert tp.peer_ranks(2, 4) == [0, 1, 3]
+    assert tp.peer_ranks(1, 2) == [0]
+    with pytest.raises(ValueError):
+        tp.peer_ranks(4, 4)
+
+
 def test_shard_layout():
     _, cache, w_uk, w_uv = _case()
     local = tp.shard_cache(cache, 2, 4)

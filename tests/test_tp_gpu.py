@@ -214,3 +214,66 @@ def test_gla2_ranks_match_the_oracle(wl):
                                       softmax_scale=wl.softmax_scale, rope_theta=wl.rope_theta)
                     for s in range(wl.batch)])
     assert_parity(got, ref, f"{wl.name} GLA-2")
+
+
+# --- the up-projection adding into every rank's out (fused all-reduce) ---------------------
+
+def _shard_params(dev, wl, rank, world, out, **kw):
+    local = tp.shard_cache(dev.cache, rank, world)
+    w_uk, w_uv = tp.shard_weights(dev.w_uk, dev.w_uv, rank, world)
+    d = local.shape[1] - synth.D_ROPE
+    p = hra.make_params(dev.q, local[:, :d], local[:, d:], dev.seq_lens, w_uk, w_uv, out, n_branch=4 // world,
+                        alpha_q=wl.alpha_q, alpha_kv=wl.alpha_kv, branch_scale=wl.sigma_o,
+                        softmax_scale=wl.softmax_scale, rope_theta=wl.rope_theta, block_table=dev.block_table,
+                        page_size=wl.page_size, seq_stride=dev.seq_stride, **kw)
+    return p, (local, w_uk, w_uv)
+
+
+@pytest.mark.parametrize("wl", [_wl("tails", (1, 31, 129, 1000)), _wl("paged64", (5, 64, 65, 700), page_size=64)],
+                         ids=lambda w: w.name)
+def test_accumulating_shards_into_one_out_gives_mlra4(wl):
+    """out_accumulate: the 4 ranks' calls add into one zeroed buffer; the sum is MLRA-4."""
+    inp = synth.make_inputs(wl)
+    dev = synth.to_device(inp)
+    out = torch.zeros(wl.batch, wl.heads, synth.D_V, dtype=torch.float32, device="cuda")
+    keep = []
+    for r in range(4):
+        p, k = _shard_params(dev, wl, r, 4, out, out_accumulate=True)
+        keep.append((hra.alloc_workspace(p), k))
+        hra.mlra_decode(p)
+        hra.check_device_status(p)
+    assert_parity(out.cpu().numpy(), oracle.decode_batch(inp, wl, form="absorbed"), f"{wl.name} accumulated")
+
+
+def test_accumulate_of_one_call_equals_the_stored_output():
+    wl = _wl("acc1", (700, 33))
+    dev = synth.to_device(synth.make_inputs(wl))
+    stored = _run_shard(dev, wl, 1, 4, 0)
+    out = torch.zeros_like(stored)
+    p, keep = _shard_params(dev, wl, 1, 4, out, out_accumulate=True)
+    ws = hra.alloc_workspace(p)
+    hra.mlra_decode(p)
+    hra.check_device_status(p)
+    assert torch.equal(out, stored)
+    del ws, keep
+
+
+@pytest.mark.parametrize("world", [4, 2])
+def test_every_rank_out_receives_every_shard(world):
+    """out_peers: rank r writes into its own out and the other ranks' (here buffers on the
+    same GPU standing in for peer memory); run in rank order, every out ends with the same
+    bits, the MLRA-4 output."""
+    wl = _wl("peers", (1, 300, 2000))
+    inp = synth.make_inputs(wl)
+    dev = synth.to_device(inp)
+    outs = [torch.zeros(wl.batch, wl.heads, synth.D_V, dtype=torch.float32, device="cuda") for _ in range(world)]
+    keep = []
+    for r in range(world):
+        p, k = _shard_params(dev, wl, r, world, outs[r], out_accumulate=True,
+                             out_peers=[outs[q] for q in tp.peer_ranks(r, world)])
+        keep.append((hra.alloc_workspace(p), k))
+        hra.mlra_decode(p)
+        hra.check_device_status(p)
+    for q in range(1, world):
+        assert torch.equal(outs[q], outs[0])
+    assert_parity(outs[0].cpu().numpy(), oracle.decode_batch(inp, wl, form="absorbed"), f"peers x{world}")
