@@ -15,7 +15,9 @@ One JSON line is printed by rank 0.
 --tp W (W = 2 or 4 for MLRA-4, 2 for MLRA-2): tensor parallelism by branch.  Rank r holds
 its W-th of the branches (cache columns + K_RoPE, W_UK / W_UV rows) and a step is its
 shard's decode followed by an NCCL all-reduce of out; run it with --gpus W.  With one GPU,
-the rank-0 shard's step is timed alone (no all-reduce).
+the rank-0 shard's step is timed alone (no all-reduce).  --fused-out replaces the NCCL
+call by the fused path: the up-projection adds into every rank's out (symmetric memory),
+bracketed by device barriers.
 """
 from __future__ import annotations
 
@@ -269,11 +271,17 @@ def run_native(args, wl, world, rank, local):
         d_c, n_branch = synth.D_C // tpw, wl.n_branch // tpw
     kv = int(lens.astype(np.int64).sum()) * (d_c + synth.D_ROPE) * 2  # cache bytes this rank reads
     stream = torch.cuda.current_stream()
-    out = torch.empty(wl.batch, wl.heads, synth.D_V, dtype=torch.float32, device="cuda")
+    peer_out = None
+    if all_reduce and args.fused_out:  # out in symmetric memory, added into by every rank
+        peer_out = hra.tp.PeerOut((wl.batch, wl.heads, synth.D_V), device=torch.device("cuda", local))
+        out = peer_out.out
+    else:
+        out = torch.empty(wl.batch, wl.heads, synth.D_V, dtype=torch.float32, device="cuda")
     p = hra.make_params(dev.q, cache[:, :d_c], cache[:, d_c:], dev.seq_lens, w_uk, w_uv, out,
                         n_branch=n_branch, alpha_q=wl.alpha_q, alpha_kv=wl.alpha_kv, branch_scale=wl.sigma_o,
                         softmax_scale=wl.softmax_scale, rope_theta=wl.rope_theta, block_table=dev.block_table,
-                        page_size=wl.page_size, seq_stride=dev.seq_stride, num_splits=args.num_splits)
+                        page_size=wl.page_size, seq_stride=dev.seq_stride, num_splits=args.num_splits,
+                        out_accumulate=peer_out is not None, out_peers=peer_out.peers if peer_out else None)
     ws = hra.alloc_workspace(p)
 
     # per-step stage events: [before absorb, before decode, before combine, after combine]
@@ -286,9 +294,14 @@ def run_native(args, wl, world, rank, local):
     assert all(h for hs in handles for h in hs), "CUDA events were not created"
 
     def call():  # one step as a user makes it: the decode call (+ the all-reduce under TP)
-        hra.mlra_decode(p, stream)
-        if all_reduce:
-            hra.tp.all_reduce_out(out)
+        if peer_out is not None:
+            peer_out.begin()
+            hra.mlra_decode(p, stream)
+            peer_out.end()
+        else:
+            hra.mlra_decode(p, stream)
+            if all_reduce:
+                hra.tp.all_reduce_out(out)
 
     for _ in range(args.warmup):
         call()
@@ -405,8 +418,12 @@ def run_native(args, wl, world, rank, local):
         achieved_tflops = flops / (decode_ms * 1e-3) / 1e12
         traffic = ncu_traffic(f"{wl.name}/tp{tpw}" if tpw else wl.name)
         if tpw:
-            parallelism = (f"tp{tpw}: branch shards + NCCL all-reduce of out" if all_reduce else
-                           f"tp{tpw}: rank 0's branch shard alone (no all-reduce)")
+            if not all_reduce:
+                parallelism = f"tp{tpw}: rank 0's branch shard alone (no all-reduce)"
+            elif peer_out is not None:
+                parallelism = f"tp{tpw}: branch shards, the up-projection adding into every rank's out (fused)"
+            else:
+                parallelism = f"tp{tpw}: branch shards + NCCL all-reduce of out"
         else:
             parallelism = f"replicas x{world}" if world > 1 else "1 GPU"
         line = {
@@ -478,6 +495,8 @@ def main():
     ap.add_argument("--no-graph", action="store_true", help="time direct calls instead of CUDA-graph replays")
     ap.add_argument("--tp", type=int, default=0, choices=[0, 2, 4],
                     help="tensor parallelism by branch over this many ranks (MLRA-4 workloads)")
+    ap.add_argument("--fused-out", action="store_true",
+                    help="with --tp on several GPUs: the up-projection adds into every rank's out")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -485,6 +504,8 @@ def main():
     wl = synth.WORKLOADS[args.workload]
     if args.tp and (wl.n_branch == 1 or wl.n_branch % args.tp != 0):
         ap.error(f"--tp {args.tp} needs whole branches per rank (MLRA-4: 2 or 4; MLRA-2: 2)")
+    if args.fused_out and not (args.tp and world == args.tp > 1):
+        ap.error("--fused-out needs --tp W on W > 1 ranks")
     if args.tp and world not in (1, args.tp):
         ap.error(f"--tp {args.tp} runs on {args.tp} ranks (or one GPU for a single shard), not {world}")
     if args.impl == "reference":
