@@ -277,3 +277,25 @@ def test_every_rank_out_receives_every_shard(world):
     for q in range(1, world):
         assert torch.equal(outs[q], outs[0])
     assert_parity(outs[0].cpu().numpy(), oracle.decode_batch(inp, wl, form="absorbed"), f"peers x{world}")
+
+
+@pytest.mark.parametrize("n_branch,world", [(4, 4), (2, 2)])
+def test_branch_shards_at_the_maximum_batch(n_branch, world):
+    """B = 1024 with zero lengths, 8 heads: shards of 128-wide (MLRA-4 / 4) and 256-wide
+    (MLRA-2 / 2) branches at the largest batch; their sum is the model's output."""
+    rng = np.random.default_rng(13)
+    lens = rng.integers(0, 300, size=1024)
+    lens[rng.integers(0, 1024, size=20)] = 0
+    wl = synth.Workload(f"maxbatch_tp{world}", n_branch, 1024, 8, int(lens.max()), lengths=tuple(int(x) for x in lens))
+    inp = synth.make_inputs(wl)
+    dev = synth.to_device(inp)
+    total = torch.zeros(wl.batch, wl.heads, synth.D_V, dtype=torch.float32, device="cuda")
+    for r in range(world):
+        local = tp.shard_cache(dev.cache, r, world, n_branch=n_branch)
+        w_uk, w_uv = tp.shard_weights(dev.w_uk, dev.w_uv, r, world, n_branch=n_branch)
+        total += _call(dev.q, local, w_uk, w_uv, dev, wl, n_branch // world, wl.sigma_o)
+    got = total.cpu().numpy()
+    zero = lens == 0
+    assert np.all(got[zero] == 0)
+    ref = oracle.decode_batch(inp, wl, seqs=[int(s) for s in np.flatnonzero(~zero)], form="absorbed")
+    assert_parity(got[~zero], ref, wl.name)
