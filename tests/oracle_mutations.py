@@ -24,6 +24,8 @@ MUTATIONS = [
     ("mlra_decode_expanded", "K = np.concatenate([K_nope, k_rope], axis=1)",
      "K = np.concatenate([K_nope, 0 * k_rope], axis=1)", "rope key dropped"),
     ("mla_decode", "1.0 / math.sqrt(d_qk) if", "1.0 / math.sqrt(d_nope) if", "MLA softmax scale"),
+    ("gla_decode", "c_kv[:, g * w:(g + 1) * w]", "c_kv[:, 0:w]", "every head group on the first latent group"),
+    ("gla_decode", "heads = slice(g * per, (g + 1) * per)", "heads = slice(0, per)", "every group on the first heads"),
 ]
 
 
