@@ -11,7 +11,8 @@ fixtures in ``tests/golden/``.  The pages print no worked numeric example of the
 own, so no pin compares against a number printed on the pages.
 """
 from .reference import (rope_rotate, mlra_decode_expanded, mlra_decode_absorbed, mla_decode, gla_decode,
+                        mlra_prefill_expanded,
                         mla_nope_key, mlra_nope_key_blocks, decode_batch)
 
-__all__ = ["rope_rotate", "mlra_decode_expanded", "mlra_decode_absorbed", "mla_decode", "gla_decode",
+__all__ = ["rope_rotate", "mlra_decode_expanded", "mlra_decode_absorbed", "mla_decode", "gla_decode", "mlra_prefill_expanded",
            "mla_nope_key", "mlra_nope_key_blocks", "decode_batch"]

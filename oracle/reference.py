@@ -223,6 +223,53 @@ def mla_decode(q, c_kv, k_rope, w_uk, w_uv, alpha_q: float = 1.0, alpha_kv: floa
     return np.stack(rows)
 
 
+def mlra_prefill_expanded(q, c_kv, k_rope, w_uk, w_uv, n_branch: int,
+                          alpha_q: float = 1.0, alpha_kv: float = 1.0,
+                          branch_scale: float | None = None,
+                          softmax_scale: float | None = None,
+                          rope_theta: float = 10000.0) -> np.ndarray:
+    """Causal multi-token (prefill) MLRA for ONE sequence, in the expanded form.
+
+    "vllbc02MLA" contrasts the two phases: prefill is compute-bound and forms the per-head
+    keys and values (the expanded form), generation is memory-bound and uses the absorbed
+    form.  The n query tokens are the last n of the sequence, at positions
+    p_j = L - n + j; query j attends to the tokens t <= p_j with the per-branch softmax of
+    "Multi-Head Low-Rank Attention" (核心方法), exactly as :func:`mlra_decode_expanded` would
+    for the first p_j + 1 tokens.
+
+    q [n, h, d_nope + d_rope] (rope part not rotated); c_kv [L, d_c]; k_rope [L, d_rope]
+    (already rotated); w_uk [h, d_c, d_nope]; w_uv [h, d_c, d_v].  Returns [n, h, d_v].
+    """
+    q, c_kv, k_rope = _f64(q), _f64(c_kv), _f64(k_rope)
+    w_uk, w_uv = _f64(w_uk), _f64(w_uv)
+    n, h, d_qk = q.shape
+    L, d_c = c_kv.shape
+    d_rope = k_rope.shape[1]
+    d_nope = d_qk - d_rope
+    if n > L:
+        raise ValueError(f"{n} query tokens but only {L} cached")
+    w = d_c // n_branch
+    tau = 1.0 / math.sqrt(d_nope + d_rope) if softmax_scale is None else softmax_scale
+    sigma = 1.0 / math.sqrt(n_branch) if branch_scale is None else branch_scale
+    pos = np.arange(L - n, L)
+    visible = np.arange(L)[None, :] <= pos[:, None]                  # [n, L] causal mask
+    out = np.zeros((n, h, w_uv.shape[2]))
+    for i in range(h):
+        q_n = alpha_q * q[:, i, :d_nope]                               # [n, d_nope]
+        q_r = np.stack([rope_rotate(q[j, i, d_nope:], int(pos[j]), rope_theta) for j in range(n)])
+        for b in range(n_branch):
+            cols = slice(b * w, (b + 1) * w)
+            K_nope = alpha_kv * (c_kv[:, cols] @ w_uk[i, cols, :])      # [L, d_nope]
+            V = alpha_kv * (c_kv[:, cols] @ w_uv[i, cols, :])           # [L, d_v]
+            score = tau * (q_n @ K_nope.T + q_r @ k_rope.T)            # [n, L]
+            score = np.where(visible, score, -np.inf)
+            score -= score.max(axis=1, keepdims=True)
+            p = np.exp(score)
+            p /= p.sum(axis=1, keepdims=True)
+            out[:, i] += p @ V
+    return sigma * out
+
+
 def gla_decode(q, c_kv, k_rope, w_uk, w_uv, n_groups: int = 2, alpha_q: float = 1.0, alpha_kv: float = 1.0,
                softmax_scale: float | None = None, rope_theta: float = 10000.0) -> np.ndarray:
     """Grouped latent attention (GLA-n) decode for ONE sequence.

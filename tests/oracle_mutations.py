@@ -26,6 +26,10 @@ MUTATIONS = [
     ("mla_decode", "1.0 / math.sqrt(d_qk) if", "1.0 / math.sqrt(d_nope) if", "MLA softmax scale"),
     ("gla_decode", "c_kv[:, g * w:(g + 1) * w]", "c_kv[:, 0:w]", "every head group on the first latent group"),
     ("gla_decode", "heads = slice(g * per, (g + 1) * per)", "heads = slice(0, per)", "every group on the first heads"),
+    ("mlra_prefill_expanded", "np.arange(L)[None, :] <= pos[:, None]", "np.arange(L)[None, :] < pos[:, None]",
+     "causal mask hides the query's own token"),
+    ("mlra_prefill_expanded", "rope_rotate(q[j, i, d_nope:], int(pos[j]), rope_theta)",
+     "rope_rotate(q[j, i, d_nope:], L - 1, rope_theta)", "every query rotated to the last position"),
 ]
 
 

@@ -129,6 +129,52 @@ def test_gla_head_reads_only_its_group():
     assert _rel(moved[2:], base[2:]) > 1e-3
 
 
+# --- the causal multi-token (prefill) form ---------------------------------------------------
+
+@pytest.mark.parametrize("n_branch", [1, 4])
+def test_prefill_rows_are_decodes_of_the_prefix(n_branch):
+    """Query j of a prefill over the last n tokens sees exactly the first p_j + 1 tokens at
+    position p_j: it equals the (pinned) decode oracle on that prefix ("vllbc02MLA":
+    prefill and generation compute the same attention).  Catches: a mask off by one, the
+    rope position of the wrong token, branch scales applied per query."""
+    rng = np.random.default_rng(21)
+    h, L, n = 3, 19, 5
+    _, c, kr, wuk, wuv = _rand_case(rng, h=h, L=L, n_branch=n_branch)
+    q = torch.from_numpy(rng.standard_normal((n, h, 192))).to(torch.bfloat16)
+    kw = dict(alpha_q=1.3, alpha_kv=0.7)
+    pre = oracle.mlra_prefill_expanded(q, c, kr, wuk, wuv, n_branch, **kw)
+    for j in range(n):
+        m = L - n + j + 1
+        ref = oracle.mlra_decode_absorbed(q[j], c[:m], kr[:m], wuk, wuv, n_branch, **kw)
+        assert _rel(pre[j], ref) < 1e-12
+
+
+def test_prefill_is_causal_and_matches_library_causal_attention():
+    """Changing tokens after a query's position leaves its row unchanged, and one branch
+    of one head equals torch's scaled_dot_product_attention with a causal (bottom-right)
+    mask on the expanded keys and values (library routine, fp64)."""
+    rng = np.random.default_rng(22)
+    h, L, n = 2, 13, 4
+    _, c, kr, wuk, wuv = _rand_case(rng, h=h, L=L, n_branch=1, bf16=False)
+    q = rng.standard_normal((n, h, 192))
+    pre = oracle.mlra_prefill_expanded(q, c, kr, wuk, wuv, 1)
+    c2 = c.copy()
+    c2[L - 2:] += 1.0  # only the last two tokens change: rows of queries before them stay
+    pre2 = oracle.mlra_prefill_expanded(q, c2, kr, wuk, wuv, 1)
+    assert np.array_equal(pre2[:n - 2], pre[:n - 2])
+    assert _rel(pre2[n - 1], pre[n - 1]) > 1e-6
+    i = 1
+    K = np.concatenate([c @ wuk[i], kr], axis=1)
+    V = c @ wuv[i]
+    pos = np.arange(L - n, L)
+    Q = np.stack([np.concatenate([q[j, i, :128], oracle.rope_rotate(q[j, i, 128:], int(pos[j]))]) for j in range(n)])
+    mask = torch.from_numpy(np.arange(L)[None, :] <= pos[:, None])
+    ref = torch.nn.functional.scaled_dot_product_attention(
+        torch.from_numpy(Q)[None], torch.from_numpy(K)[None], torch.from_numpy(V)[None], attn_mask=mask[None],
+        scale=1 / math.sqrt(192))[0].numpy()
+    assert _rel(pre[:, i], ref) < 1e-12
+
+
 # --- RoPE --------------------------------------------------------------------------------
 
 def test_rope_relative_position():
