@@ -432,11 +432,9 @@ def run_native(args, wl, world, rank, local):
             "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": step_ms, "us_per_step": step_ms * 1e3,
             "higher_is_better": True, "scaling": "strong" if tpw else "weak", "vs_baseline": None,
-            "dtype": "bf16" if wl.n_branch == 4 else "f16",
-            "precision": ("bf16 inputs; bf16 tensor-core operands, the absorbed query as two bf16 terms; "
-                          "fp32 accumulate, softmax, combine") if wl.n_branch == 4 else
-                         ("bf16 inputs; fp16 tensor-core operands (cache tile converted in shared memory); "
-                          "fp32 accumulate, softmax, combine"),
+            "dtype": "f16",
+            "precision": "bf16 inputs; fp16 tensor-core operands (absorbed query fp16, cache tile converted "
+                         "bf16 -> fp16 in shared memory, P fp16); fp32 accumulate, softmax, combine",
             "data": "synthetic",
             "config": dict(workload_config(wl, lens, tpw), parallelism=parallelism,
                            num_splits=args.num_splits or f"auto (SMs/{d_c // 128})",

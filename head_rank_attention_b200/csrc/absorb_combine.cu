@@ -10,8 +10,7 @@
 // contiguous nope dims: K-major), D in 256 TMEM columns.  bf16 x bf16
 // products are exact in the fp32 accumulator, so this equals the fp32 definition up to
 // summation order.  A thread of the epilogue owns one sequence and 32 consecutive latent
-// columns at a time, so q~ (fp16, or the two-term bf16 split the MLRA-4 kernel uses) is
-// written with 16-byte stores.  The same threads rotate q_rope to position L-1.  The
+// columns at a time, so q~ (fp16) is written with 16-byte stores.  The same threads rotate q_rope to position L-1.  The
 // branch structure needs no special case: branch b's absorbed query is columns
 // [b*w, (b+1)*w) of the same d_c-vector (W_UK^(b),(i) is the matching row block).
 //
@@ -50,29 +49,14 @@ struct AbsorbCfg {
   static constexpr int THREADS = 256;
 };
 
-// 32 consecutive fp32 values -> q~ at dst (fp16, or bf16 hi at dst and lo at dst + lo_off).
-__device__ __forceinline__ void store_q32(const AbsorbArgs& a, long long dst, long long lo_off, const float* x) {
-  if (a.two_term) {
-    __nv_bfloat16* hi = reinterpret_cast<__nv_bfloat16*>(a.q_tilde);
+// 32 consecutive fp32 values -> fp16 q~ at dst.
+__device__ __forceinline__ void store_q32(const AbsorbArgs& a, long long dst, const float* x) {
 #pragma unroll
-    for (int v = 0; v < 4; ++v) {
-      __align__(16) __nv_bfloat16 h8[8], l8[8];
+  for (int v = 0; v < 4; ++v) {
+    __align__(16) __half h8[8];
 #pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        h8[u] = __float2bfloat16_rn(x[8 * v + u]);
-        l8[u] = __float2bfloat16_rn(x[8 * v + u] - __bfloat162float(h8[u]));
-      }
-      *reinterpret_cast<uint4*>(hi + dst + 8 * v) = *reinterpret_cast<const uint4*>(h8);
-      *reinterpret_cast<uint4*>(hi + lo_off + dst + 8 * v) = *reinterpret_cast<const uint4*>(l8);
-    }
-  } else {
-#pragma unroll
-    for (int v = 0; v < 4; ++v) {
-      __align__(16) __half h8[8];
-#pragma unroll
-      for (int u = 0; u < 8; ++u) h8[u] = __float2half_rn(x[8 * v + u]);
-      *reinterpret_cast<uint4*>(a.q_tilde + dst + 8 * v) = *reinterpret_cast<const uint4*>(h8);
-    }
+    for (int u = 0; u < 8; ++u) h8[u] = __float2half_rn(x[8 * v + u]);
+    *reinterpret_cast<uint4*>(a.q_tilde + dst + 8 * v) = *reinterpret_cast<const uint4*>(h8);
   }
 }
 
@@ -144,14 +128,11 @@ absorb_tc_kernel(const __grid_constant__ CUtensorMap map_wuk, const __grid_const
   // Everything above reads only inputs of the call; what follows writes the workspace,
   // which the previous call's kernels read, so it waits for them.
   grid_dep_wait();
-  if (blockIdx.x == 0 && blockIdx.y == 0 && blockIdx.z == 0) {
-    if (threadIdx.x < 4) a.status[threadIdx.x] = 0;  // fresh per call
-    if (warp == 3) tile_prefix_warp(a.seq_lens, a.batch, a.tile_tokens, a.tile_prefix);
-  }
+  if (blockIdx.x == 0 && blockIdx.y == 0 && blockIdx.z == 0 && warp == 3)
+    tile_prefix_warp(a.seq_lens, a.batch, a.tile_tokens, a.tile_prefix);
   const int r = 32 * (warp & 3) + lane;  // sequence within the chunk = TMEM lane
   const int s = s0 + r;
   const int part = warp >> 2;            // columns [256 nh + 128 part, +128); rope pairs [16 part, +16)
-  const long long lo_off = static_cast<long long>(a.batch) * a.heads * (dc + 64);
   const long long row = (static_cast<long long>(s) * a.heads + i) * (dc + 64);
   if (s < a.batch && nh == 0) {
     // RoPE of the query's rope part at position L-1, while the loads and MMAs run: pair
@@ -178,7 +159,7 @@ absorb_tc_kernel(const __grid_constant__ CUtensorMap map_wuk, const __grid_const
       y2[u] = fmaf(a1, sn, a2 * cs);
     }
     // rotated pair halves: elements [16 part, +16) and [32 + 16 part, +16) of the rope part
-    {  // fp16 in both modes (the two-term query's rope slot of the hi array)
+    {
 #pragma unroll
       for (int h2 = 0; h2 < 2; ++h2) {
         const float* y = h2 == 0 ? y1 : y2;
@@ -209,7 +190,7 @@ absorb_tc_kernel(const __grid_constant__ CUtensorMap map_wuk, const __grid_const
         float x[32];
 #pragma unroll
         for (int u = 0; u < 32; ++u) x[u] = scale * __uint_as_float(v[u]);
-        store_q32(a, row + k0, lo_off, x);
+        store_q32(a, row + k0, x);
       }
     }
   }

@@ -12,9 +12,8 @@ namespace hra {
 struct AbsorbArgs {
   const __nv_bfloat16* q;     // [B, h, 192]
   const int32_t* seq_lens;    // [B]
-  __half* q_tilde;            // out: fp16 [B, h, d_c + 64], or (two_term) bf16 hi then bf16 lo, each [B, h, d_c + 64]
-  int two_term;               // 1: store q~ as bf16 hi + bf16 lo (128-wide-branch kernel); 0: fp16
-  int* status;                // cleared by this kernel (first kernel of a call)
+  __half* q_tilde;            // out: fp16 [B, h, d_c + 64]: absorbed latent query | rotated rope part
+  int* status;                // device status word (expired waits)
   int* tile_prefix;           // out: [B + 1] exclusive prefix of decode tiles per sequence
   int tile_tokens;            // decode tile size (tokens)
   int batch, heads;

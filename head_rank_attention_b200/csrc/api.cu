@@ -38,6 +38,9 @@ hra_status cuda_fail(cudaError_t e, const char* what) {
 }
 
 constexpr uint64_t kDefaultWaitLimitUs = 1000000;  // 1 s per device-side wait
+// Smallest limit a call may set: far above the time any one tile's copy, conversion or
+// MMAs take, so that a wait only expires when the pipeline is really stuck.
+constexpr uint64_t kMinWaitLimitUs = 10000;  // 10 ms
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 size_t round256(size_t x) { return (x + 255) & ~size_t(255); }
@@ -134,8 +137,8 @@ hra_status make_plan(const hra_decode_params* p, Plan* plan) {
   plan->slots = static_cast<long long>(plan->groups) + p->batch;
   const size_t slices = static_cast<size_t>(p->d_c) / 128;
   size_t off = 256;  // device status word
-  plan->q_tilde = off;  // up to two terms of [B, h, d_c + 64]
-  off = round256(off + 2 * static_cast<size_t>(p->batch) * p->num_heads * (p->d_c + 64) * sizeof(__half));
+  plan->q_tilde = off;  // fp16 [B, h, d_c + 64]
+  off = round256(off + static_cast<size_t>(p->batch) * p->num_heads * (p->d_c + 64) * sizeof(__half));
   plan->o_part = off;
   off = round256(off + static_cast<size_t>(plan->slots) * slices * 128 * 128 * sizeof(float));
   plan->ml_part = off;
@@ -214,6 +217,11 @@ hra_status run_decode(const hra_decode_params* p, cudaStream_t stream) {
   };
   cudaError_t e = mark(0);
   if (e != cudaSuccess) return cuda_fail(e, "stage event");
+  // The status word starts each call at zero.  It is cleared in stream order before any
+  // kernel of the call runs, so that no block of any kernel can record an expired wait
+  // before the clear lands (a memset allocates nothing).
+  e = cudaMemsetAsync(status, 0, 4 * sizeof(int), stream);
+  if (e != cudaSuccess) return cuda_fail(e, "status clear");
 
   hra::AbsorbArgs ab{};
   ab.q = static_cast<const __nv_bfloat16*>(p->q);
@@ -226,7 +234,6 @@ hra_status run_decode(const hra_decode_params* p, cudaStream_t stream) {
   ab.alpha_kv = p->alpha_kv;
   ab.rope_theta = p->rope_theta;
   ab.d_c = dc;
-  ab.two_term = dc / p->n_branch == 128 ? 1 : 0;  // 128-wide branches: the two-term split kernel
   ab.tile_prefix = tile_prefix;
   ab.tile_tokens = hra::decode_tile_tokens(dc / p->n_branch);
   // Programmatic dependent launch lets each kernel start while the previous one drains;
@@ -251,7 +258,8 @@ hra_status run_decode(const hra_decode_params* p, cudaStream_t stream) {
   da.o_part = o_part;
   da.ml_part = ml_part;
   da.status = status;
-  da.wait_limit_ns = 1000ull * (p->wait_limit > 0 ? static_cast<uint64_t>(p->wait_limit) : kDefaultWaitLimitUs);
+  const uint64_t limit_us = p->wait_limit > 0 ? static_cast<uint64_t>(p->wait_limit) : kDefaultWaitLimitUs;
+  da.wait_limit_ns = 1000ull * (limit_us < kMinWaitLimitUs ? kMinWaitLimitUs : limit_us);
   if ((e = mark(1)) != cudaSuccess) return cuda_fail(e, "stage event");
   e = hra::launch_decode_kernel(p->n_branch, map_ckv, map_krope, da, plan.groups, stream, pdl);
   if (e != cudaSuccess) return cuda_fail(e, "decode launch");

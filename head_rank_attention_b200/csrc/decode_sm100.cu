@@ -226,7 +226,7 @@ decode_kernel(const __grid_constant__ CUtensorMap map_ckv, const __grid_constant
       if (ok && !warp_wait(&empty[k % STAGES], (k / STAGES) & 1, limit, abort_flag, status, 2)) ok = false;
       if (!ok) {  // aborted: wait (bounded, ignoring the abort flag) for the copy itself
         volatile int never = 0;
-        warp_wait(&full[k % STAGES], (k / STAGES) & 1, limit, &never, status, 3);
+        warp_wait(&full[k % STAGES], (k / STAGES) & 1, kDrainNs, &never, status, 3);
       }
     }
   } else if (warp == 13) {
@@ -271,11 +271,11 @@ decode_kernel(const __grid_constant__ CUtensorMap map_ckv, const __grid_constant
         tc_fence_after();
         issue_pv<C>(tiles_addr, tmem, pv_done, empty, it - 1, j1 - 1 == j0, pv_box);
       }
-      if (!ok) {  // drain: let every MMA issued so far finish before TMEM is released
-        umma_commit(drain);
-        volatile int never = 0;
-        mbar_wait(drain, 0, limit, &never, status, 14);
-      }
+      // drain: every MMA issued so far completes before TMEM is released (bounded by
+      // kDrainNs, whatever the abort flag says)
+      umma_commit(drain);
+      volatile int never = 0;
+      mbar_wait(drain, 0, kDrainNs, &never, status, 14);
     }
   } else if (warp >= 8) {
     // ------------------------------------------------------------------ bf16 -> fp16

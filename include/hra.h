@@ -32,12 +32,9 @@
  * Bounded device waits that expire write a status word in the workspace, read back
  * by hra_check_device_status().
  * Numerics: bf16 inputs, fp32 accumulation; softmax, combine and up-projection in fp32.
- * 128-wide branches (d_c / n_branch = 128): the tensor cores read the latent
- * part of the cache as stored, against
- * the absorbed query carried as two bf16 terms (hi + lo, ~16 significant bits); the rope
- * part (query and K_RoPE tile) is scored in fp16, so |K_RoPE values| must stay below 65504.
- * 256- and 512-wide branches: the cache tile is converted to fp16 in shared memory and the
- * query is fp16, so |cache values| must stay below 65504.
+ * The decode kernels convert each cache tile to fp16 in shared memory (exact for bf16
+ * values of fp16's range) and score it against the absorbed query in fp16; the softmax
+ * weights P are fp16 in the P.V product.  |cache values| must stay below 65504.
  * Stream order: the kernels of a call are chained with programmatic dependent launch, so
  * a call may begin (set-up, loads of its inputs) while the previous call on the stream
  * drains; it touches the workspace only once that call has completed.
@@ -117,7 +114,9 @@ typedef struct {
   size_t workspace_bytes;
   int num_splits;       /* KV splits = groups of d_c/128 CTAs streaming disjoint token
                            ranges; 0 = one group per d_c/128 SMs of the current device    */
-  int wait_limit;       /* microseconds one device-side wait may last; 0 = 1 s           */
+  int wait_limit;       /* microseconds one device-side wait may last; 0 = 1 s.  Values
+                           below 10000 (10 ms) are raised to 10 ms, far above the time any
+                           one tile's copy, conversion or MMAs take                     */
   void* const* stage_events; /* optional, NULL = none: 4 caller-owned cudaEvent_t recorded on
                                 `stream` before absorption, before the split-KV decode, before
                                 the combine/up-projection and after it (per-stage timing)    */

@@ -73,7 +73,7 @@ def test_workspace_size_formula(d_c, n_branch, splits):
     n = hra.workspace_size(p)
     slots, slices = splits + 2, d_c // 128
     expect = 256
-    expect = -(-(expect + 2 * 2 * 128 * (d_c + 64) * 2) // 256) * 256  # q~ as up to two 16-bit terms
+    expect = -(-(expect + 2 * 128 * (d_c + 64) * 2) // 256) * 256  # fp16 q~
     expect = -(-(expect + slots * slices * 128 * 128 * 4) // 256) * 256
     expect = -(-(expect + slots * slices * 128 * 8) // 256) * 256
     expect = -(-(expect + 2 * 128 * 2 * d_c * 2) // 256) * 256  # merged latent as two bf16 terms
