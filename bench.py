@@ -12,6 +12,13 @@ Multi-GPU (torchrun, one rank per GPU): every rank decodes its own replica batch
 path has no exchange step); value = all ranks' KV bytes / max-over-ranks step time.
 One JSON line is printed by rank 0.
 
+--gpus N without torchrun: bench.py launches itself as N ranks (torch.distributed.run,
+rendezvous on 127.0.0.1); under torchrun, --gpus must equal WORLD_SIZE.
+
+--gla 2 (MLA workloads): a rank of GLA-2, MLA's latent split into two 256-wide groups
+with half of the heads each (2.5 d_h of cache per token and rank); with one GPU, rank 0's
+call is timed alone, with 2 GPUs the ranks' outs are gathered over heads.
+
 --tp W (W = 2 or 4 for MLRA-4, 2 for MLRA-2): tensor parallelism by branch.  Rank r holds
 its W-th of the branches (cache columns + K_RoPE, W_UK / W_UV rows) and a step is its
 shard's decode followed by an NCCL all-reduce of out; run it with --gpus W.  With one GPU,
@@ -150,10 +157,11 @@ class ClockSampler:
                 "samples": len(clks), "source": "NVML, 2 ms period, timed region only"}
 
 
-def time_oracle_sample(wl: synth.Workload, n_seqs: int, n_heads: int, tp_world: int = 0):
+def time_oracle_sample(wl: synth.Workload, n_seqs: int, n_heads: int, tp_world: int = 0, gla: int = 0):
     """Run the fp64 oracle (the expanded definition) on n_seqs x n_heads outputs of the
-    workload (of its rank-0 branch shard under tp_world-way tensor parallelism, if set);
-    return (seconds, the sample's share of the step, threads used, sequences, heads)."""
+    workload (of its rank-0 branch shard under tp_world-way tensor parallelism, or of rank
+    0's group under GLA, if set); return (seconds, the sample's share of the step, threads
+    used, sequences, heads)."""
     import oracle
     from head_rank_attention_b200 import tp
     try:
@@ -172,19 +180,31 @@ def time_oracle_sample(wl: synth.Workload, n_seqs: int, n_heads: int, tp_world: 
         rows = {s: tp.shard_cache(r, 0, tp_world, n_branch) for s, r in rows.items()}
         w_uk, w_uv = tp.shard_weights(w_uk, w_uv, 0, tp_world, n_branch)
         d_c, n_branch = synth.D_C // tp_world, wl.n_branch // tp_world
+    n_heads_rank = wl.heads
+    if gla:  # group 0: latent columns [0, 512 / gla) and the first h / gla heads
+        per = wl.heads // gla
+        rows = {s: tp.shard_cache(r, 0, gla, n_branch=gla) for s, r in rows.items()}
+        w_uk, w_uv = w_uk[:per, :synth.D_C // gla], w_uv[:per, :synth.D_C // gla]
+        q = q[:, :per]
+        heads = heads[:per]
+        d_c, n_branch, n_heads_rank = synth.D_C // gla, 1, per
     t0 = time.perf_counter()
     for s in seqs:
         r = rows[s]
         oracle.mlra_decode_expanded(q[s], r[:, :d_c], r[:, d_c:], w_uk, w_uv, n_branch,
-                                    alpha_q=wl.alpha_q, alpha_kv=wl.alpha_kv, branch_scale=wl.sigma_o,
+                                    alpha_q=wl.alpha_q, alpha_kv=wl.alpha_kv,
+                                    branch_scale=1.0 if gla else wl.sigma_o,
                                     softmax_scale=wl.softmax_scale, rope_theta=wl.rope_theta, heads=heads)
     dt = time.perf_counter() - t0
     # the sample's share of the full step, by cached tokens x heads
-    frac = (sum(int(lens[s]) for s in seqs) * len(heads)) / (int(lens.sum()) * wl.heads)
+    frac = (sum(int(lens[s]) for s in seqs) * len(heads)) / (int(lens.sum()) * n_heads_rank)
     return dt, frac, threads, len(seqs), len(heads)
 
 
-def workload_config(wl: synth.Workload, lens, tp_world: int = 0) -> dict:
+def workload_config(wl: synth.Workload, lens, tp_world: int = 0, gla: int = 0) -> dict:
+    if gla:
+        return dict(workload_config(wl, lens), variant=f"GLA-{gla} rank", d_c=512 // gla, heads=wl.heads // gla,
+                    branch_scale=1.0, gla_rank=f"1 of {gla} latent groups, {wl.heads // gla} of {wl.heads} heads")
     return {"workload": wl.name, "variant": {1: "MLA", 2: "MLRA-2", 4: "MLRA-4"}[wl.n_branch],
             "batch": wl.batch, "heads": wl.heads, "seq_len": wl.seq_len,
             "seq_len_min": wl.seq_len_min, "total_tokens": int(np.asarray(lens, dtype=np.int64).sum()),
@@ -209,6 +229,19 @@ def job_tbs(bytes_per_rank: int, world: int, ms_per_step: float) -> float:
     return world * bytes_per_rank / (ms_per_step * 1e-3) / 1e12
 
 
+def self_launch(n: int) -> int:
+    """Run this script as n ranks (one per GPU) under torch.distributed.run on 127.0.0.1;
+    returns the launcher's exit status."""
+    import socket
+    with socket.socket(socket.AF_INET, socket.SOCK_STREAM) as sk:
+        sk.bind(("127.0.0.1", 0))
+        port = sk.getsockname()[1]
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", f"--nproc-per-node={n}",
+           "--master-addr", "127.0.0.1", f"--master-port={port}", str(pathlib.Path(__file__).resolve()),
+           *sys.argv[1:]]
+    return subprocess.call(cmd)
+
+
 def dist_setup():
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -221,14 +254,15 @@ def run_reference(args, wl, world, rank):
         return
     lens = synth.seq_lens(wl)
     tpw = getattr(args, "tp", 0)
-    d_c = synth.D_C // tpw if tpw else synth.D_C
+    gla = getattr(args, "gla", 0)
+    d_c = synth.D_C // tpw if tpw else synth.D_C // gla if gla else synth.D_C
     kv = int(np.asarray(lens, dtype=np.int64).sum()) * (d_c + synth.D_ROPE) * 2
     for _ in range(args.warmup):
-        time_oracle_sample(wl, 1, 1, tpw)
+        time_oracle_sample(wl, 1, 1, tpw, gla)
     times = []
     frac = threads = None
     for _ in range(args.steps):
-        dt, frac, threads, ns, nh = time_oracle_sample(wl, args.ref_seqs, args.ref_heads, tpw)
+        dt, frac, threads, ns, nh = time_oracle_sample(wl, args.ref_seqs, args.ref_heads, tpw, gla)
         times.append(dt / frac)  # extrapolated seconds per full decode step
     step_s = statistics.mean(times)
     value = kv / step_s / 1e12
@@ -237,7 +271,7 @@ def run_reference(args, wl, world, rank):
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "TB/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": step_s * 1e3,
             "us_per_step": step_s * 1e6, "higher_is_better": True, "scaling": "strong" if tpw else "weak",
-            "vs_baseline": None, "dtype": "f64", "data": "synthetic", "config": workload_config(wl, lens, tpw),
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic", "config": workload_config(wl, lens, tpw, gla),
             "cpu_baseline": {"value": value, "unit": "TB/s", "cores": threads, "kind": "oracle", "sample": sample},
             "e2e": {"value": value, "unit": "TB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
@@ -260,6 +294,23 @@ def run_native(args, wl, world, rank, local):
     d_c, n_branch = synth.D_C, wl.n_branch
     cache, w_uk, w_uv = dev.cache, dev.w_uk, dev.w_uv
     host_cache, host_wuk, host_wuv = inp.cache, inp.w_uk, inp.w_uv
+    gla = getattr(args, "gla", 0)
+    heads = wl.heads
+    q_dev, host_q = dev.q, inp.q
+    branch_scale = wl.sigma_o
+    if gla:  # this rank's GLA-2 group: latent columns [256 g, +256), K_RoPE, heads [h g / 2, +h / 2)
+        g = rank if world == gla else 0
+        per = wl.heads // gla
+        hsl = slice(g * per, (g + 1) * per)
+        cols = slice(g * (synth.D_C // gla), (g + 1) * (synth.D_C // gla))
+        cache = hra.tp.shard_cache(dev.cache, g, gla, n_branch=gla)
+        host_cache = hra.tp.shard_cache(inp.cache, g, gla, n_branch=gla)
+        w_uk, w_uv = dev.w_uk[hsl, cols].contiguous(), dev.w_uv[hsl, cols].contiguous()
+        host_wuk, host_wuv = inp.w_uk[hsl, cols].contiguous(), inp.w_uv[hsl, cols].contiguous()
+        q_dev, host_q = dev.q[:, hsl].contiguous(), inp.q[:, hsl].contiguous()
+        dev.cache = dev.w_uk = dev.w_uv = None
+        torch.cuda.empty_cache()
+        d_c, n_branch, heads, branch_scale = synth.D_C // gla, 1, per, 1.0
     if tpw:  # this rank's branch shard (rank 0's when one GPU stands alone)
         shard = rank if world == tpw else 0
         cache = hra.tp.shard_cache(dev.cache, shard, tpw, wl.n_branch)
@@ -276,9 +327,11 @@ def run_native(args, wl, world, rank, local):
         peer_out = hra.tp.PeerOut((wl.batch, wl.heads, synth.D_V), device=torch.device("cuda", local))
         out = peer_out.out
     else:
-        out = torch.empty(wl.batch, wl.heads, synth.D_V, dtype=torch.float32, device="cuda")
-    p = hra.make_params(dev.q, cache[:, :d_c], cache[:, d_c:], dev.seq_lens, w_uk, w_uv, out,
-                        n_branch=n_branch, alpha_q=wl.alpha_q, alpha_kv=wl.alpha_kv, branch_scale=wl.sigma_o,
+        out = torch.empty(wl.batch, heads, synth.D_V, dtype=torch.float32, device="cuda")
+    gathered = (torch.empty(world, wl.batch, heads, synth.D_V, dtype=torch.float32, device="cuda")
+                if gla and world > 1 else None)
+    p = hra.make_params(q_dev, cache[:, :d_c], cache[:, d_c:], dev.seq_lens, w_uk, w_uv, out,
+                        n_branch=n_branch, alpha_q=wl.alpha_q, alpha_kv=wl.alpha_kv, branch_scale=branch_scale,
                         softmax_scale=wl.softmax_scale, rope_theta=wl.rope_theta, block_table=dev.block_table,
                         page_size=wl.page_size, seq_stride=dev.seq_stride, num_splits=args.num_splits,
                         out_accumulate=peer_out is not None, out_peers=peer_out.peers if peer_out else None)
@@ -302,6 +355,8 @@ def run_native(args, wl, world, rank, local):
             hra.mlra_decode(p, stream)
             if all_reduce:
                 hra.tp.all_reduce_out(out)
+            elif gathered is not None:  # GLA-2: the ranks' heads side by side
+                torch.distributed.all_gather_into_tensor(gathered, out)
 
     for _ in range(args.warmup):
         call()
@@ -314,7 +369,7 @@ def run_native(args, wl, world, rank, local):
 
     # Inputs smaller than twice the L2 (126 MB) would stay cached between steps: flush it
     # by writing a 512 MB buffer before every timed step.
-    step_bytes = kv + sum(t.numel() * t.element_size() for t in (dev.q, w_uk, w_uv))
+    step_bytes = kv + sum(t.numel() * t.element_size() for t in (q_dev, w_uk, w_uv))
     step_bytes_all = step_bytes + out.numel() * 4
     flush = torch.zeros(128 << 20, dtype=torch.float32, device="cuda") if step_bytes < (252 << 20) else None
 
@@ -322,7 +377,7 @@ def run_native(args, wl, world, rank, local):
     # dependent launch), replayed from a CUDA graph of one call unless --no-graph, so that
     # host-side launch work does not bound the short configurations.
     graph = None
-    if not args.no_graph and not all_reduce:
+    if not args.no_graph and not all_reduce and gathered is None:
         graph = torch.cuda.CUDAGraph()
         with torch.cuda.graph(graph):
             hra.mlra_decode(p, torch.cuda.current_stream())
@@ -384,12 +439,12 @@ def run_native(args, wl, world, rank, local):
     decode_ms = float(stage_ms[:, 1].mean())
 
     # end to end through the C ABI with host buffers: H2D of every input, decode, D2H of out
-    pin = {k: v.pin_memory() for k, v in dict(q=inp.q, cache=host_cache, seq_lens=inp.seq_lens,
+    pin = {k: v.pin_memory() for k, v in dict(q=host_q, cache=host_cache, seq_lens=inp.seq_lens,
                                                w_uk=host_wuk, w_uv=host_wuv).items()}
     if inp.block_table is not None:
         pin["block_table"] = inp.block_table.pin_memory()
     host_out = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
-    dmap = dict(q=dev.q, cache=cache, seq_lens=dev.seq_lens, w_uk=w_uk, w_uv=w_uv,
+    dmap = dict(q=q_dev, cache=cache, seq_lens=dev.seq_lens, w_uk=w_uk, w_uv=w_uv,
                 block_table=dev.block_table)
     h2d = sum(t.numel() * t.element_size() for t in pin.values())
     d2h = host_out.numel() * host_out.element_size()
@@ -406,18 +461,38 @@ def run_native(args, wl, world, rank, local):
     torch.cuda.synchronize()
     e2e_ms = e0.elapsed_time(e1) / e2e_steps
     hra.check_device_status(p, stream)
+    # the same with the cache and weights resident (as in serving): per step only the
+    # query, the lengths (and block table) go host -> device and out comes back
+    per_step = [k for k in ("q", "seq_lens", "block_table") if k in pin]
+    h2d_res = sum(pin[k].numel() * pin[k].element_size() for k in per_step)
+    r_steps = max(1, args.steps)
+    barrier()
+    r0, r1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    r0.record(stream)
+    for _ in range(r_steps):
+        for k in per_step:
+            dmap[k].copy_(pin[k], non_blocking=True)
+        call()
+        host_out.copy_(out, non_blocking=True)
+    r1.record(stream)
+    torch.cuda.synchronize()
+    res_ms = r0.elapsed_time(r1) / r_steps
+    hra.check_device_status(p, stream)
 
     step_ms = elapsed_ms / args.steps
-    step_ms, e2e_ms, decode_ms = max_over_ranks([step_ms, e2e_ms, decode_ms], world, "cuda")
+    step_ms, e2e_ms, decode_ms, res_ms = max_over_ranks([step_ms, e2e_ms, decode_ms, res_ms], world, "cuda")
     clocks = clk.summary()
 
     if rank == 0:
         pk, pk_src = peaks()
         achieved_gbs = kv / (decode_ms * 1e-3) / 1e9
-        flops = tensor_flops_per_token(n_branch, wl.heads, d_c) * int(lens.astype(np.int64).sum())
+        flops = tensor_flops_per_token(n_branch, heads, d_c) * int(lens.astype(np.int64).sum())
         achieved_tflops = flops / (decode_ms * 1e-3) / 1e12
         traffic = ncu_traffic(f"{wl.name}/tp{tpw}" if tpw else wl.name)
-        if tpw:
+        if gla:
+            parallelism = (f"gla{gla}: head-and-latent groups, outs gathered over heads" if world == gla
+                           else f"gla{gla}: rank 0's group alone (no gather)")
+        elif tpw:
             if not all_reduce:
                 parallelism = f"tp{tpw}: rank 0's branch shard alone (no all-reduce)"
             elif peer_out is not None:
@@ -436,7 +511,7 @@ def run_native(args, wl, world, rank, local):
             "precision": "bf16 inputs; fp16 tensor-core operands (absorbed query fp16, cache tile converted "
                          "bf16 -> fp16 in shared memory, P fp16); fp32 accumulate, softmax, combine",
             "data": "synthetic",
-            "config": dict(workload_config(wl, lens, tpw), parallelism=parallelism,
+            "config": dict(workload_config(wl, lens, tpw, gla), parallelism=parallelism,
                            num_splits=args.num_splits or f"auto (SMs/{d_c // 128})",
                            timing="CUDA-graph replays of one call" if graph_used else "direct calls",
                            **({} if flush is None else
@@ -452,17 +527,23 @@ def run_native(args, wl, world, rank, local):
                          "bound": "hbm", "achieved": achieved_gbs,
                          "peak": pk["hbm_gbs"], "unit": "GB/s", "frac": achieved_gbs / pk["hbm_gbs"],
                          "peak_source": pk_src, "traffic": traffic,
-                         "bytes_per_launch": kv},
+                         "bytes_per_launch": kv,
+                         # the same bytes over the whole step (all four kernels)
+                         "frac_step": kv / (step_ms * 1e-3) / 1e9 / pk["hbm_gbs"]},
             "roofline_tensor": {"achieved": achieved_tflops, "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
                                 "frac": achieved_tflops / pk["bf16_tflops"],
                                 "note": "algorithmic FLOPs (rope scored once, one query term) over the bf16 dense peak"},
             "clocks": clocks,
             "e2e": {"value": job_tbs(kv, world, e2e_ms), "unit": "TB/s", "ms_per_step": e2e_ms,
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": e2e_steps},
+            "e2e_resident_cache": {"value": job_tbs(kv, world, res_ms), "unit": "TB/s", "ms_per_step": res_ms,
+                                   "h2d_bytes_per_step": h2d_res, "d2h_bytes_per_step": d2h, "steps": r_steps,
+                                   "note": "cache and weights resident in HBM; per step the query, lengths "
+                                           "(and block table) are copied in and out is copied back"},
             "gpu_launches": 4 * args.steps,  # absorb, decode, merge, up-projection per step
         }
         if world == 1 and not args.no_cpu_baseline:
-            dt, frac, threads, ns, nh = time_oracle_sample(wl, args.cpu_seqs, args.cpu_heads, tpw)
+            dt, frac, threads, ns, nh = time_oracle_sample(wl, args.cpu_seqs, args.cpu_heads, tpw, gla)
             cpu_step = dt / frac
             line["cpu_baseline"] = {
                 "value": kv / cpu_step / 1e12, "unit": "TB/s", "cores": threads, "kind": "oracle",
@@ -495,15 +576,27 @@ def main():
                     help="tensor parallelism by branch over this many ranks (MLRA-4 workloads)")
     ap.add_argument("--fused-out", action="store_true",
                     help="with --tp on several GPUs: the up-projection adds into every rank's out")
+    ap.add_argument("--gla", type=int, default=0, choices=[0, 2],
+                    help="a rank of GLA-2 on an MLA workload (2 latent groups, half the heads each)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
+    if args.gpus < 1:
+        ap.error("--gpus must be >= 1")
+    if "WORLD_SIZE" not in os.environ and args.gpus > 1:
+        sys.exit(self_launch(args.gpus))
     world, rank, local = dist_setup()
+    if world != args.gpus:
+        ap.error(f"--gpus {args.gpus} but WORLD_SIZE={world}: run one rank per GPU")
     wl = synth.WORKLOADS[args.workload]
     if args.tp and (wl.n_branch == 1 or wl.n_branch % args.tp != 0):
         ap.error(f"--tp {args.tp} needs whole branches per rank (MLRA-4: 2 or 4; MLRA-2: 2)")
     if args.fused_out and not (args.tp and world == args.tp > 1):
         ap.error("--fused-out needs --tp W on W > 1 ranks")
+    if args.gla and (wl.n_branch != 1 or args.tp):
+        ap.error("--gla 2 takes an MLA workload and no --tp")
+    if args.gla and world not in (1, args.gla):
+        ap.error(f"--gla {args.gla} runs on {args.gla} ranks (or one GPU for a single group), not {world}")
     if args.tp and world not in (1, args.tp):
         ap.error(f"--tp {args.tp} runs on {args.tp} ranks (or one GPU for a single shard), not {world}")
     if args.impl == "reference":

@@ -104,3 +104,48 @@ def test_tensor_flops_per_token_of_a_shard():
     import bench
     assert bench.tensor_flops_per_token(4, 128) == 2176 * 128
     assert bench.tensor_flops_per_token(1, 128, 128) == (2 * 192 + 2 * 128) * 128
+
+
+def _bench_cmd(*extra):
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    return [sys.executable, os.path.join(root, "bench.py"), "--impl", "reference", "--steps", "1", "--warmup", "3",
+            "--ref-seqs", "1", "--ref-heads", "1", "--workload", "small_mlra4_h16_t2k", *extra]
+
+
+def test_gpus_flag_launches_that_many_ranks():
+    """bench.py --gpus 2 run by hand (no torchrun) launches itself as two ranks; rank 0
+    alone prints the line, which reports both ranks."""
+    import json
+    import subprocess
+    env = {k: v for k, v in os.environ.items() if k not in ("WORLD_SIZE", "RANK", "LOCAL_RANK")}
+    r = subprocess.run(_bench_cmd("--gpus", "2"), env=env, capture_output=True, text=True, timeout=600)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [json.loads(l) for l in r.stdout.splitlines() if l.startswith("{")]
+    assert len(lines) == 1
+    assert lines[0]["n_gpus"] == 2 and lines[0]["impl"] == "reference"
+
+
+def test_gpus_flag_must_match_the_launcher():
+    """Under a launcher, --gpus must equal WORLD_SIZE."""
+    import subprocess
+    env = dict(os.environ, WORLD_SIZE="1", RANK="0", LOCAL_RANK="0")
+    r = subprocess.run(_bench_cmd("--gpus", "2"), env=env, capture_output=True, text=True, timeout=300)
+    assert r.returncode == 2 and "WORLD_SIZE=1" in r.stderr
+
+
+def test_reference_arm_for_a_gla2_rank_reports_the_group():
+    """--gla 2 on an MLA workload: rank 0's group is 256 latent columns, the rope key and
+    half of the heads; 2.5 d_h of cache per token."""
+    import argparse
+    import json
+
+    import bench
+    import synth
+    wl = synth.Workload("gla_small", 1, 1, 16, 2048)
+    out = io.StringIO()
+    with contextlib.redirect_stdout(out):
+        bench.run_reference(argparse.Namespace(steps=1, warmup=3, ref_seqs=1, ref_heads=1, tp=0, gla=2), wl, 1, 0)
+    line = json.loads(out.getvalue())
+    assert line["config"]["d_c"] == 256 and line["config"]["heads"] == 8
+    assert line["config"]["variant"] == "GLA-2 rank"
+    assert line["value"] == pytest.approx(2048 * (256 + 64) * 2 / (line["ms_per_step"] * 1e-3) / 1e12)
