@@ -15,6 +15,10 @@ One JSON line is printed by rank 0.
 --gpus N without torchrun: bench.py launches itself as N ranks (torch.distributed.run,
 rendezvous on 127.0.0.1); under torchrun, --gpus must equal WORLD_SIZE.
 
+--cache int8 (MLRA-4 workloads and their branch shards): the latent cache is int8 with one
+fp32 scale per token and 128-column block (K_RoPE stays bf16): 656 instead of 1152 bytes per
+token.
+
 --gla 2 (MLA workloads): a rank of GLA-2, MLA's latent split into two 256-wide groups
 with half of the heads each (2.5 d_h of cache per token and rank); with one GPU, rank 0's
 call is timed alone, with 2 GPUs the ranks' outs are gathered over heads.
@@ -157,7 +161,8 @@ class ClockSampler:
                 "samples": len(clks), "source": "NVML, 2 ms period, timed region only"}
 
 
-def time_oracle_sample(wl: synth.Workload, n_seqs: int, n_heads: int, tp_world: int = 0, gla: int = 0):
+def time_oracle_sample(wl: synth.Workload, n_seqs: int, n_heads: int, tp_world: int = 0, gla: int = 0,
+                       int8: bool = False):
     """Run the fp64 oracle (the expanded definition) on n_seqs x n_heads outputs of the
     workload (of its rank-0 branch shard under tp_world-way tensor parallelism, or of rank
     0's group under GLA, if set); return (seconds, the sample's share of the step, threads
@@ -188,10 +193,15 @@ def time_oracle_sample(wl: synth.Workload, n_seqs: int, n_heads: int, tp_world: 
         q = q[:, :per]
         heads = heads[:per]
         d_c, n_branch, n_heads_rank = synth.D_C // gla, 1, per
+    if int8:  # the sample's latent rows as the int8 cache stands for them
+        rows = {s: (oracle.dequantize_int8_blocks(*synth.quantize_int8_blocks(r[:, :d_c])), r[:, d_c:])
+                for s, r in rows.items()}
+    else:
+        rows = {s: (r[:, :d_c], r[:, d_c:]) for s, r in rows.items()}
     t0 = time.perf_counter()
     for s in seqs:
-        r = rows[s]
-        oracle.mlra_decode_expanded(q[s], r[:, :d_c], r[:, d_c:], w_uk, w_uv, n_branch,
+        c, kr = rows[s]
+        oracle.mlra_decode_expanded(q[s], c, kr, w_uk, w_uv, n_branch,
                                     alpha_q=wl.alpha_q, alpha_kv=wl.alpha_kv,
                                     branch_scale=1.0 if gla else wl.sigma_o,
                                     softmax_scale=wl.softmax_scale, rope_theta=wl.rope_theta, heads=heads)
@@ -256,13 +266,15 @@ def run_reference(args, wl, world, rank):
     tpw = getattr(args, "tp", 0)
     gla = getattr(args, "gla", 0)
     d_c = synth.D_C // tpw if tpw else synth.D_C // gla if gla else synth.D_C
-    kv = int(np.asarray(lens, dtype=np.int64).sum()) * (d_c + synth.D_ROPE) * 2
+    int8 = getattr(args, "cache", "bf16") == "int8"
+    per_token = d_c + 2 * synth.D_ROPE + 4 * (d_c // 128) if int8 else (d_c + synth.D_ROPE) * 2
+    kv = int(np.asarray(lens, dtype=np.int64).sum()) * per_token
     for _ in range(args.warmup):
-        time_oracle_sample(wl, 1, 1, tpw, gla)
+        time_oracle_sample(wl, 1, 1, tpw, gla, int8)
     times = []
     frac = threads = None
     for _ in range(args.steps):
-        dt, frac, threads, ns, nh = time_oracle_sample(wl, args.ref_seqs, args.ref_heads, tpw, gla)
+        dt, frac, threads, ns, nh = time_oracle_sample(wl, args.ref_seqs, args.ref_heads, tpw, gla, int8)
         times.append(dt / frac)  # extrapolated seconds per full decode step
     step_s = statistics.mean(times)
     value = kv / step_s / 1e12
@@ -271,7 +283,9 @@ def run_reference(args, wl, world, rank):
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "TB/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": step_s * 1e3,
             "us_per_step": step_s * 1e6, "higher_is_better": True, "scaling": "strong" if tpw else "weak",
-            "vs_baseline": None, "dtype": "f64", "data": "synthetic", "config": workload_config(wl, lens, tpw, gla),
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": dict(workload_config(wl, lens, tpw, gla), cache="int8" if int8 else "bf16",
+                           cache_bytes_per_token=per_token),
             "cpu_baseline": {"value": value, "unit": "TB/s", "cores": threads, "kind": "oracle", "sample": sample},
             "e2e": {"value": value, "unit": "TB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
@@ -320,7 +334,19 @@ def run_native(args, wl, world, rank, local):
         dev.cache = dev.w_uk = dev.w_uv = None
         torch.cuda.empty_cache()
         d_c, n_branch = synth.D_C // tpw, wl.n_branch // tpw
-    kv = int(lens.astype(np.int64).sum()) * (d_c + synth.D_ROPE) * 2  # cache bytes this rank reads
+    int8 = args.cache == "int8"
+    ckv_scale = None
+    if int8:  # quantise this rank's latent columns (input preparation, outside the timed region)
+        q8, ckv_scale = synth.quantize_int8_blocks(cache[:, :d_c])
+        host_q8, host_scale = q8.cpu(), ckv_scale.cpu()  # the same bytes for the end-to-end leg
+        krope_dev = cache[:, d_c:].contiguous()
+        host_krope = host_cache[:, d_c:].contiguous()
+        cache = None
+        torch.cuda.empty_cache()
+        per_token = d_c + 2 * synth.D_ROPE + 4 * (d_c // 128)
+    else:
+        per_token = (d_c + synth.D_ROPE) * 2
+    kv = int(lens.astype(np.int64).sum()) * per_token  # cache bytes this rank reads
     stream = torch.cuda.current_stream()
     peer_out = None
     if all_reduce and args.fused_out:  # out in symmetric memory, added into by every rank
@@ -330,7 +356,8 @@ def run_native(args, wl, world, rank, local):
         out = torch.empty(wl.batch, heads, synth.D_V, dtype=torch.float32, device="cuda")
     gathered = (torch.empty(world, wl.batch, heads, synth.D_V, dtype=torch.float32, device="cuda")
                 if gla and world > 1 else None)
-    p = hra.make_params(q_dev, cache[:, :d_c], cache[:, d_c:], dev.seq_lens, w_uk, w_uv, out,
+    ckv_view, krope_view = (q8, krope_dev) if int8 else (cache[:, :d_c], cache[:, d_c:])
+    p = hra.make_params(q_dev, ckv_view, krope_view, dev.seq_lens, w_uk, w_uv, out, ckv_scale=ckv_scale,
                         n_branch=n_branch, alpha_q=wl.alpha_q, alpha_kv=wl.alpha_kv, branch_scale=branch_scale,
                         softmax_scale=wl.softmax_scale, rope_theta=wl.rope_theta, block_table=dev.block_table,
                         page_size=wl.page_size, seq_stride=dev.seq_stride, num_splits=args.num_splits,
@@ -439,12 +466,15 @@ def run_native(args, wl, world, rank, local):
     decode_ms = float(stage_ms[:, 1].mean())
 
     # end to end through the C ABI with host buffers: H2D of every input, decode, D2H of out
-    pin = {k: v.pin_memory() for k, v in dict(q=host_q, cache=host_cache, seq_lens=inp.seq_lens,
+    host_inputs = (dict(q=host_q, ckv=host_q8, scale=host_scale, krope=host_krope) if int8 else
+                   dict(q=host_q, cache=host_cache))
+    pin = {k: v.pin_memory() for k, v in dict(**host_inputs, seq_lens=inp.seq_lens,
                                                w_uk=host_wuk, w_uv=host_wuv).items()}
     if inp.block_table is not None:
         pin["block_table"] = inp.block_table.pin_memory()
     host_out = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
-    dmap = dict(q=q_dev, cache=cache, seq_lens=dev.seq_lens, w_uk=w_uk, w_uv=w_uv,
+    dmap = dict(q=q_dev, seq_lens=dev.seq_lens, w_uk=w_uk, w_uv=w_uv,
+                **(dict(ckv=q8, scale=ckv_scale, krope=krope_dev) if int8 else dict(cache=cache)),
                 block_table=dev.block_table)
     h2d = sum(t.numel() * t.element_size() for t in pin.values())
     d2h = host_out.numel() * host_out.element_size()
@@ -512,6 +542,8 @@ def run_native(args, wl, world, rank, local):
                          "bf16 -> fp16 in shared memory, P fp16); fp32 accumulate, softmax, combine",
             "data": "synthetic",
             "config": dict(workload_config(wl, lens, tpw, gla), parallelism=parallelism,
+                           cache=("int8, one fp32 scale per token and 128-column block; K_RoPE bf16" if int8
+                                  else "bf16"), cache_bytes_per_token=per_token,
                            num_splits=args.num_splits or f"auto (SMs/{d_c // 128})",
                            timing="CUDA-graph replays of one call" if graph_used else "direct calls",
                            **({} if flush is None else
@@ -543,7 +575,7 @@ def run_native(args, wl, world, rank, local):
             "gpu_launches": 4 * args.steps,  # absorb, decode, merge, up-projection per step
         }
         if world == 1 and not args.no_cpu_baseline:
-            dt, frac, threads, ns, nh = time_oracle_sample(wl, args.cpu_seqs, args.cpu_heads, tpw, gla)
+            dt, frac, threads, ns, nh = time_oracle_sample(wl, args.cpu_seqs, args.cpu_heads, tpw, gla, int8)
             cpu_step = dt / frac
             line["cpu_baseline"] = {
                 "value": kv / cpu_step / 1e12, "unit": "TB/s", "cores": threads, "kind": "oracle",
@@ -576,6 +608,8 @@ def main():
                     help="tensor parallelism by branch over this many ranks (MLRA-4 workloads)")
     ap.add_argument("--fused-out", action="store_true",
                     help="with --tp on several GPUs: the up-projection adds into every rank's out")
+    ap.add_argument("--cache", default="bf16", choices=["bf16", "int8"],
+                    help="latent cache format (int8: MLRA-4 workloads and their branch shards)")
     ap.add_argument("--gla", type=int, default=0, choices=[0, 2],
                     help="a rank of GLA-2 on an MLA workload (2 latent groups, half the heads each)")
     args = ap.parse_args()
@@ -593,6 +627,8 @@ def main():
         ap.error(f"--tp {args.tp} needs whole branches per rank (MLRA-4: 2 or 4; MLRA-2: 2)")
     if args.fused_out and not (args.tp and world == args.tp > 1):
         ap.error("--fused-out needs --tp W on W > 1 ranks")
+    if args.cache == "int8" and (args.gla or (512 // wl.n_branch) != 128):
+        ap.error("--cache int8 takes an MLRA-4 workload (128-wide branches)")
     if args.gla and (wl.n_branch != 1 or args.tp):
         ap.error("--gla 2 takes an MLA workload and no --tp")
     if args.gla and world not in (1, args.gla):

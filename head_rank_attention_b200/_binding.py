@@ -19,6 +19,7 @@ HRA_ERR_CUDA = -4
 HRA_ERR_DEVICE_TIMEOUT = -5
 HRA_BF16 = 0
 HRA_F32 = 1
+HRA_INT8 = 2
 
 STATUS_NAMES = {0: "HRA_OK", -1: "HRA_ERR_INVALID_ARG", -2: "HRA_ERR_UNSUPPORTED", -3: "HRA_ERR_WORKSPACE",
                 -4: "HRA_ERR_CUDA", -5: "HRA_ERR_DEVICE_TIMEOUT"}
@@ -51,6 +52,7 @@ class HraDecodeParams(ctypes.Structure):
         ("num_splits", ctypes.c_int), ("wait_limit", ctypes.c_int),
         ("stage_events", ctypes.c_void_p),
         ("out_accumulate", ctypes.c_int), ("n_out_peers", ctypes.c_int), ("out_peers", ctypes.c_void_p),
+        ("cache_dtype", ctypes.c_int), ("ckv_scale", ctypes.c_void_p), ("ckv_scale_stride", ctypes.c_int64),
     ]
 
 
@@ -110,11 +112,12 @@ def make_params(q, ckv, krope, seq_lens, w_uk, w_uv, out, workspace=None, *, n_b
                 softmax_scale: float = 0.0, rope_theta: float = 10000.0, block_table=None,
                 page_size: int = 0, seq_stride: int = 0, cache_rows: Optional[int] = None,
                 num_splits: int = 0, wait_limit: int = 0, out_accumulate: bool = False,
-                out_peers=None) -> HraDecodeParams:
+                out_peers=None, ckv_scale=None) -> HraDecodeParams:
     """Fill hra_decode_params from torch tensors (shapes/dtypes as documented in hra.h).
 
     ckv / krope are 2-D row views of the cache (e.g. cache[:, :512], cache[:, 512:]);
-    their row strides become ckv_stride / krope_stride.  out_peers: device addresses (ints)
+    their row strides become ckv_stride / krope_stride.  An int8 ckv selects the quantised
+    cache: ckv_scale is then the fp32 [rows, d_c / 128] view of its block scales.  out_peers: device addresses (ints)
     or tensors of other ranks' out buffers for out_accumulate (the array is kept alive on
     the returned object).
     """
@@ -125,6 +128,11 @@ def make_params(q, ckv, krope, seq_lens, w_uk, w_uv, out, workspace=None, *, n_b
     p.d_c, p.d_rope, p.d_nope, p.d_v = int(ckv.shape[1]), int(krope.shape[1]), int(q.shape[2]) - int(krope.shape[1]), int(w_uv.shape[2])
     p.q, p.ckv, p.krope = _ptr(q), _ptr(ckv), _ptr(krope)
     p.ckv_stride, p.krope_stride = int(ckv.stride(0)), int(krope.stride(0))
+    if ckv.dtype == torch.int8:
+        if ckv_scale is None:
+            raise ValueError("an int8 cache needs ckv_scale")
+        p.cache_dtype = HRA_INT8
+        p.ckv_scale, p.ckv_scale_stride = _ptr(ckv_scale), int(ckv_scale.stride(0))
     p.cache_rows = int(ckv.shape[0]) if cache_rows is None else int(cache_rows)
     p.seq_lens = _ptr(seq_lens)
     p.block_table = _ptr(block_table)

@@ -118,6 +118,20 @@ hra_status validate(const hra_decode_params* p) {
         return fail(HRA_ERR_INVALID_ARG, "out_peers[%d] is NULL or not 16-byte aligned", k);
   }
   if (p->wait_limit < 0) return fail(HRA_ERR_INVALID_ARG, "wait_limit=%d must be >= 0", p->wait_limit);
+  if (p->cache_dtype == HRA_INT8) {
+    if (p->d_c / p->n_branch != 128)
+      return fail(HRA_ERR_UNSUPPORTED, "an int8 cache is supported for 128-wide branches (d_c / n_branch = %d)",
+                  p->d_c / p->n_branch);
+    if (p->ckv_scale == nullptr || (reinterpret_cast<uintptr_t>(p->ckv_scale) & 3u) != 0)
+      return fail(HRA_ERR_INVALID_ARG, "ckv_scale is NULL or not 4-byte aligned");
+    if (p->ckv_scale_stride < p->d_c / 128)
+      return fail(HRA_ERR_INVALID_ARG, "ckv_scale_stride=%lld must be >= d_c / 128", (long long)p->ckv_scale_stride);
+    if (p->ckv_stride % 16 != 0)
+      return fail(HRA_ERR_INVALID_ARG, "ckv_stride=%lld bytes must be a multiple of 16 for an int8 cache",
+                  (long long)p->ckv_stride);
+  } else if (p->cache_dtype != HRA_BF16) {
+    return fail(HRA_ERR_INVALID_ARG, "cache_dtype=%d (HRA_BF16 or HRA_INT8)", (int)p->cache_dtype);
+  }
   if (!std::isfinite(p->alpha_q) || !std::isfinite(p->alpha_kv) || !std::isfinite(p->branch_scale) ||
       !std::isfinite(p->softmax_scale) || !(p->rope_theta > 0.f) || !std::isfinite(p->rope_theta))
     return fail(HRA_ERR_INVALID_ARG, "scales must be finite and rope_theta > 0");
@@ -154,9 +168,10 @@ hra_status make_plan(const hra_decode_params* p, Plan* plan) {
 std::once_flag g_encode_once;
 PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
 
-// 2-D bf16 view [rows, inner] with row stride `stride_elems`, boxes of 64 x box_rows, 128-byte swizzle.
+// 2-D view [rows, inner] with row stride `stride_elems`, boxes of box_inner x box_rows, 128-byte
+// swizzle; bf16 elements, or bytes (int8 cache) with byte8 = true.
 hra_status encode_map(CUtensorMap* map, const void* base, int64_t inner, int64_t rows, int64_t stride_elems,
-                      int box_rows) {
+                      int box_rows, bool byte8 = false, int box_inner = 64) {
   std::call_once(g_encode_once, [] {
     void* fn = nullptr;
     cudaDriverEntryPointQueryResult q{};
@@ -166,10 +181,11 @@ hra_status encode_map(CUtensorMap* map, const void* base, int64_t inner, int64_t
   });
   if (g_encode == nullptr) return fail(HRA_ERR_CUDA, "cuTensorMapEncodeTiled entry point unavailable");
   const cuuint64_t dims[2] = {static_cast<cuuint64_t>(inner), static_cast<cuuint64_t>(rows)};
-  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(stride_elems) * 2};
-  const cuuint32_t box[2] = {64, static_cast<cuuint32_t>(box_rows)};
+  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(stride_elems) * (byte8 ? 1 : 2)};
+  const cuuint32_t box[2] = {static_cast<cuuint32_t>(box_inner), static_cast<cuuint32_t>(box_rows)};
   const cuuint32_t estr[2] = {1, 1};
-  CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+  CUresult r = g_encode(map, byte8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
+                        const_cast<void*>(base), dims, strides, box, estr,
                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return fail(HRA_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
@@ -209,7 +225,10 @@ hra_status run_decode(const hra_decode_params* p, cudaStream_t stream) {
   if ((st = encode_map(&map_olat, o_lat, dc, 2 * static_cast<int64_t>(h) * B, dc, hra::upproj_seq_chunk())) !=
       HRA_OK)
     return st;
-  if ((st = encode_map(&map_ckv, p->ckv, dc, p->cache_rows, p->ckv_stride, 32)) != HRA_OK) return st;
+  const bool int8 = p->cache_dtype == HRA_INT8;
+  // int8: one 128-byte box per 128-wide branch and 32 rows; bf16: 64-column boxes
+  if ((st = encode_map(&map_ckv, p->ckv, dc, p->cache_rows, p->ckv_stride, 32, int8, int8 ? 128 : 64)) != HRA_OK)
+    return st;
   if ((st = encode_map(&map_krope, p->krope, 64, p->cache_rows, p->krope_stride, 32)) != HRA_OK) return st;
 
   auto mark = [&](int k) -> cudaError_t {
@@ -260,6 +279,9 @@ hra_status run_decode(const hra_decode_params* p, cudaStream_t stream) {
   da.status = status;
   const uint64_t limit_us = p->wait_limit > 0 ? static_cast<uint64_t>(p->wait_limit) : kDefaultWaitLimitUs;
   da.wait_limit_ns = 1000ull * (limit_us < kMinWaitLimitUs ? kMinWaitLimitUs : limit_us);
+  da.cache_int8 = int8 ? 1 : 0;
+  da.ckv_scale = int8 ? p->ckv_scale : nullptr;
+  da.scale_stride = int8 ? p->ckv_scale_stride : 0;
   if ((e = mark(1)) != cudaSuccess) return cuda_fail(e, "stage event");
   e = hra::launch_decode_kernel(p->n_branch, map_ckv, map_krope, da, plan.groups, stream, pdl);
   if (e != cudaSuccess) return cuda_fail(e, "decode launch");
@@ -311,6 +333,16 @@ __global__ void wait_timeout_selftest_kernel(int* status, uint64_t limit_ns) {
 namespace hra {
 // Lets other entry points of this library report through hra_last_error().
 void set_last_error(const char* msg) { g_last_error = msg; }
+// Workspace bytes of a call, with the status of the validation or device query that failed.
+hra_status workspace_bytes(const hra_decode_params* p, size_t* bytes) {
+  *bytes = 0;
+  hra_status st = validate(p);
+  if (st != HRA_OK) return st;
+  Plan plan;
+  if ((st = make_plan(p, &plan)) != HRA_OK) return st;
+  *bytes = plan.total;
+  return HRA_OK;
+}
 }  // namespace hra
 
 extern "C" {

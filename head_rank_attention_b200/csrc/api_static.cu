@@ -11,13 +11,16 @@
 //   * Every GPU that loads this library holds the array (kStaticScratchBytes) until the
 //     process exits.
 //   * All calls on a device share it and it keeps the previous call's contents.  What
-//     must start at zero -- the status word -- is cleared by the first kernel of every
-//     call; everything else is written before it is read.
+//     must start at zero -- the status word -- is cleared at the start of every call (a
+//     memset on the stream, which allocates nothing); everything else is written before
+//     it is read.
 //   * Calls that overlap on the GPU (concurrent streams, or host threads launching on
 //     different streams) race on the array and give wrong results; serialize them.
 //   * The first call on a device looks the array's device address up
 //     (cudaGetSymbolAddress) with that device current; make that first call before any
-//     stream capture.
+//     stream capture.  The address is kept for the life of the process, so the library
+//     must not be used across a device reset (cudaDeviceReset or a primary-context
+//     teardown), after which the array is mapped anew.
 //   * Expired device waits are recorded in the array's status word, which
 //     hra_check_device_status cannot reach; launch and argument errors are returned.
 #include <cuda_runtime.h>
@@ -30,7 +33,8 @@
 #include "hra.h"
 
 namespace hra {
-void set_last_error(const char* msg);  // api.cu
+void set_last_error(const char* msg);                           // api.cu
+hra_status workspace_bytes(const hra_decode_params* p, size_t* bytes);  // api.cu
 }  // namespace hra
 
 namespace {
@@ -52,9 +56,11 @@ hra_status static_fail(hra_status st, const std::string& msg) {
 
 extern "C" HRA_API hra_status mlra_decode_static(const hra_decode_params* p, void* stream) {
   if (p == nullptr) return static_fail(HRA_ERR_INVALID_ARG, "params is NULL");
-  // Size check first: it needs no device.  hra_workspace_size validates the parameters.
-  const size_t need = hra_workspace_size(p);
-  if (need == 0) return HRA_ERR_INVALID_ARG;  // hra_workspace_size recorded the reason
+  // Size check first.  It validates the parameters and, unless num_splits > 0, queries the
+  // current device's SM count (the default split count depends on it).
+  size_t need = 0;
+  const hra_status st = hra::workspace_bytes(p, &need);
+  if (st != HRA_OK) return st;  // the reason is recorded for hra_last_error
   if (need > kStaticScratchBytes) {
     char buf[256];
     snprintf(buf, sizeof(buf),

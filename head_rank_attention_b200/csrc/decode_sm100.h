@@ -27,6 +27,9 @@ struct DecodeArgs {
   float2* ml_part;            // fp32 [slots, d_c / 128, 128] pairs: (running max in log2 units, row sum)
   int* status;                // device status word
   uint64_t wait_limit_ns;     // global-time budget of one device-side wait
+  int cache_int8;             // 1: the latent cache is int8 with per-(row, 128-column block) scales
+  const float* ckv_scale;     // fp32 scales of row r at ckv_scale + r * scale_stride (int8 cache)
+  long long scale_stride;
 };
 
 // Cache row of the 32-row chunk that starts at token `tok` of sequence s (length L):

@@ -56,6 +56,7 @@ struct SplitCfg {
   static constexpr int BOXES = 3;                 // 64-column boxes per tile: 2 latent + 1 rope
   static constexpr int BOX_BYTES = NT * 128;
   static constexpr int STAGE_BYTES = BOXES * BOX_BYTES;
+  static constexpr int STAGE_BYTES_I8 = 2 * BOX_BYTES;  // int8 cache: 128 bytes of latent + the rope box per row
   static constexpr int CHUNKS = NT / 32;          // TMA row chunks per box
   static constexpr int TMEM_O = 0;
   static constexpr int TMEM_S = 128;              // two buffers of NT columns
@@ -70,7 +71,8 @@ struct SplitCfg {
   static constexpr int THREADS = 32 * (WARP_PV + 1);                // 480
   static constexpr int BAR_BYTES = 512;
   static constexpr int RED_BYTES = (2 * 2 * 128 + 2 * 128) * 4;
-  static constexpr int MISC_BYTES = BAR_BYTES + RED_BYTES + 4 * (kMaxBatch + 1);
+  static constexpr int SCALE_BYTES = STAGES * NT * 4;  // int8 cache: each stage's 128 row scales
+  static constexpr int MISC_BYTES = BAR_BYTES + RED_BYTES + SCALE_BYTES + 4 * (kMaxBatch + 1);
   static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + MISC_BYTES;
   static_assert(TMEM_QR + 32 <= TMEM_COLS, "TMEM budget");
   static_assert(SMEM_BYTES <= 232448, "shared memory budget");
@@ -122,6 +124,8 @@ __device__ __forceinline__ void drain_mmas(uint64_t* bar, volatile int* never, i
   mbar_wait(bar, 0, kDrainNs, never, status, where);
 }
 
+// INT8: the latent cache is int8 with per-(row, 128-column block) scales (a.cache_int8 = 1).
+template <bool INT8>
 __global__ void __launch_bounds__(SplitCfg::THREADS, 1)
 decode_split_kernel(const __grid_constant__ CUtensorMap map_ckv, const __grid_constant__ CUtensorMap map_krope,
                     const DecodeArgs a) {
@@ -145,7 +149,8 @@ decode_split_kernel(const __grid_constant__ CUtensorMap map_ckv, const __grid_co
   volatile int* never_flag = abort_flag + 1;  // stays 0: exit-path waits ignore the abort flag
   float* red_max = reinterpret_cast<float*>(misc + C::BAR_BYTES);  // [2 buf][2 half][128]
   float* red_l = red_max + 2 * 2 * 128;                              // [2 half][128]
-  int* prefix = reinterpret_cast<int*>(misc + C::BAR_BYTES + C::RED_BYTES);
+  float* row_scale = reinterpret_cast<float*>(misc + C::BAR_BYTES + C::RED_BYTES);  // [STAGES][NT]
+  int* prefix = reinterpret_cast<int*>(misc + C::BAR_BYTES + C::RED_BYTES + C::SCALE_BYTES);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -210,11 +215,23 @@ decode_split_kernel(const __grid_constant__ CUtensorMap map_ckv, const __grid_co
       const int s = seq_of_tile(prefix, B, t);
       return cache_chunk_row(a, s, (t - prefix[s]) * NT + 32 * (lane % C::CHUNKS));
     };
+    // int8 cache: the 32 block scales of this lane's chunk (0 for rows past the cache),
+    // loaded one batch ahead like the rows themselves
+    auto chunk_scales = [&](int crow, float* sc) {
+#pragma unroll
+      for (int i = 0; i < 32; ++i)
+        sc[i] = crow + i < a.cache_rows ? a.ckv_scale[(static_cast<long long>(crow) + i) * a.scale_stride + slice]
+                                        : 0.f;
+    };
     int rows = chunk_row(0);
+    float sc[INT8 ? 32 : 1];
+    if constexpr (INT8) chunk_scales(rows, sc);
     int issued = 0;
     bool ok = true;
     for (int it0 = 0; ok && it0 < ntiles; it0 += TPB) {
       const int rows_next = chunk_row(it0 + TPB);
+      float sc_next[INT8 ? 32 : 1];
+      if constexpr (INT8) chunk_scales(rows_next, sc_next);
       for (int k = 0; k < TPB && it0 + k < ntiles; ++k) {
         const int it = it0 + k, stage = it % STAGES;
         if (it >= STAGES && !warp_wait(&empty[stage], ((it / STAGES) + 1) & 1, limit, abort_flag, status, 1)) {
@@ -224,25 +241,38 @@ decode_split_kernel(const __grid_constant__ CUtensorMap map_ckv, const __grid_co
         int y[C::CHUNKS];
 #pragma unroll
         for (int r = 0; r < C::CHUNKS; ++r) y[r] = __shfl_sync(kAll, rows, k * C::CHUNKS + r);
+        if (INT8 && lane / C::CHUNKS == k) {
+          // the stage's row scales, written before the stage is armed (the arrive below
+          // releases them to the converters' wait on full)
+          float4* dst = reinterpret_cast<float4*>(row_scale + stage * NT + 32 * (lane % C::CHUNKS));
+#pragma unroll
+          for (int i = 0; i < 8; ++i) dst[i] = make_float4(sc[4 * i], sc[4 * i + 1], sc[4 * i + 2], sc[4 * i + 3]);
+        }
+        __syncwarp();
         if (lane == 0) {
-          mbar_arrive_expect_tx(&full[stage], C::STAGE_BYTES);
+          mbar_arrive_expect_tx(&full[stage], INT8 ? C::STAGE_BYTES_I8 : C::STAGE_BYTES);
           uint8_t* dst = tiles + stage * C::STAGE_BYTES;
 #pragma unroll
           for (int r = 0; r < C::CHUNKS; ++r) {
+            if constexpr (INT8) {  // the branch's 128 int8 columns land where latent box 1 goes
+              tma_load_2d(dst + C::BOX_BYTES + r * 4096, &map_ckv, &full[stage], slice * C::W, y[r], policy);
+            } else {
 #pragma unroll
-            for (int d = 0; d < C::BOXES; ++d) {
-              void* box = dst + d * C::BOX_BYTES + r * 4096;
-              if (d < C::BOXES - 1)
-                tma_load_2d(box, &map_ckv, &full[stage], slice * C::W + 64 * d, y[r], policy);
-              else
-                tma_load_2d(box, &map_krope, &full[stage], 0, y[r], policy);
+              for (int d = 0; d < C::BOXES - 1; ++d)
+                tma_load_2d(dst + d * C::BOX_BYTES + r * 4096, &map_ckv, &full[stage], slice * C::W + 64 * d, y[r],
+                            policy);
             }
+            tma_load_2d(dst + 2 * C::BOX_BYTES + r * 4096, &map_krope, &full[stage], 0, y[r], policy);
           }
         }
         __syncwarp();
         issued = it + 1;
       }
       rows = rows_next;
+      if constexpr (INT8) {
+#pragma unroll
+        for (int i = 0; i < 32; ++i) sc[i] = sc_next[i];
+      }
     }
     for (int k = max(0, issued - STAGES); k < issued; ++k) {  // every stage must come back
       if (ok && !warp_wait(&empty[k % STAGES], (k / STAGES) & 1, limit, abort_flag, status, 2)) ok = false;
@@ -318,7 +348,10 @@ decode_split_kernel(const __grid_constant__ CUtensorMap map_ckv, const __grid_co
     // Rewrites each arrived stage (3 boxes x 128 rows x 128 B, swizzled 16-byte chunks
     // within each row) as fp16 in place.  Rows at or past the sequence end hold whatever
     // the cache holds there; they are zeroed so that neither their scores (masked by the
-    // softmax) nor 0 * Inf / NaN in P.V can reach O.
+    // softmax) nor 0 * Inf / NaN in P.V can reach O.  An int8 cache arrives as one 128-byte
+    // row per token in latent box 1's place; thread ct then expands row ct: it reads the
+    // row's 8 chunks, scales them by the row's block scale and writes 16 fp16 chunks over
+    // boxes 0 and 1 (and converts the row's rope chunks).
     const int ct = threadIdx.x - 32 * C::SOFTMAX_WARPS;  // 0..127
     TileCursor cc;
     cc.init(prefix, B, t_begin, t_end, s_first);
@@ -331,21 +364,71 @@ decode_split_kernel(const __grid_constant__ CUtensorMap map_ckv, const __grid_co
       }
       const int stage = it % STAGES;
       const int n_valid = min(NT, L - (cc.j - prefix[cc.s]) * NT);
-      if (!warp_wait(&full[stage], (it / STAGES) & 1, limit, abort_flag, status, 20)) break;
-      uint4* r = reinterpret_cast<uint4*>(tiles + stage * C::STAGE_BYTES);
-#pragma unroll 4
-      for (int e = ct; e < C::STAGE_BYTES / 16; e += 32 * C::CONV_WARPS) {
-        const int row = (e >> 3) & (NT - 1);
-        uint4 v = r[e];
-        if (row < n_valid) {
-          v.x = bf16x2_to_f16x2(v.x);
-          v.y = bf16x2_to_f16x2(v.y);
-          v.z = bf16x2_to_f16x2(v.z);
-          v.w = bf16x2_to_f16x2(v.w);
-        } else {
-          v = make_uint4(0u, 0u, 0u, 0u);
+      uint8_t* st = tiles + stage * C::STAGE_BYTES;
+      if constexpr (INT8) {
+        const int r = ct;
+        if (!warp_wait(&full[stage], (it / STAGES) & 1, limit, abort_flag, status, 20)) break;
+        const float scale = row_scale[stage * NT + r];  // written by the producer with the stage
+        const int sw = r & 7;
+        const __half2 s2 = __float2half2_rn(scale);
+        // Two halves of 4 chunks: the first half writes box 0 only; the second reads its
+        // chunks (and the first half has read its own) before box 1 is overwritten.
+#pragma unroll 1
+        for (int c0 = 0; c0 < 8; c0 += 4) {
+          uint4 raw[4];
+#pragma unroll
+          for (int c = 0; c < 4; ++c)
+            raw[c] = *reinterpret_cast<const uint4*>(st + C::BOX_BYTES + r * 128 + (((c0 + c) ^ sw) << 4));
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {  // int8 columns [16 (c0+c), +16) -> fp16 chunks 2 (c0+c), 2 (c0+c) + 1
+            const uint32_t wv[4] = {raw[c].x, raw[c].y, raw[c].z, raw[c].w};
+            uint32_t h[8];
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              const uint2 f = i8x4_to_f16x4(wv[q], s2);
+              h[2 * q] = f.x;
+              h[2 * q + 1] = f.y;
+            }
+#pragma unroll
+            for (int k = 0; k < 2; ++k) {
+              const int j = 2 * (c0 + c) + k;
+              const uint4 v = r < n_valid ? make_uint4(h[4 * k], h[4 * k + 1], h[4 * k + 2], h[4 * k + 3])
+                                          : make_uint4(0u, 0u, 0u, 0u);
+              *reinterpret_cast<uint4*>(st + (j >> 3) * C::BOX_BYTES + r * 128 + (((j & 7) ^ sw) << 4)) = v;
+            }
+          }
         }
-        r[e] = v;
+        uint4* rope = reinterpret_cast<uint4*>(st + 2 * C::BOX_BYTES + r * 128);
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+          uint4 v = rope[c];
+          if (r < n_valid) {
+            v.x = bf16x2_to_f16x2(v.x);
+            v.y = bf16x2_to_f16x2(v.y);
+            v.z = bf16x2_to_f16x2(v.z);
+            v.w = bf16x2_to_f16x2(v.w);
+          } else {
+            v = make_uint4(0u, 0u, 0u, 0u);
+          }
+          rope[c] = v;
+        }
+      } else {
+        if (!warp_wait(&full[stage], (it / STAGES) & 1, limit, abort_flag, status, 20)) break;
+        uint4* r = reinterpret_cast<uint4*>(st);
+#pragma unroll 4
+        for (int e = ct; e < C::STAGE_BYTES / 16; e += 32 * C::CONV_WARPS) {
+          const int row = (e >> 3) & (NT - 1);
+          uint4 v = r[e];
+          if (row < n_valid) {
+            v.x = bf16x2_to_f16x2(v.x);
+            v.y = bf16x2_to_f16x2(v.y);
+            v.z = bf16x2_to_f16x2(v.z);
+            v.w = bf16x2_to_f16x2(v.w);
+          } else {
+            v = make_uint4(0u, 0u, 0u, 0u);
+          }
+          r[e] = v;
+        }
       }
       fence_proxy_async_smem();
       warp_arrive(&conv[stage]);
@@ -504,11 +587,11 @@ int decode_split_tile_tokens() { return SplitCfg::NT; }
 cudaError_t launch_decode_split_kernel(const CUtensorMap& map_ckv, const CUtensorMap& map_krope,
                                        const DecodeArgs& a, int groups, cudaStream_t stream, bool pdl) {
   using C = SplitCfg;
-  cudaError_t e = cudaFuncSetAttribute(decode_split_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       C::SMEM_BYTES);
+  auto kern = a.cache_int8 ? decode_split_kernel<true> : decode_split_kernel<false>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
   if (e != cudaSuccess) return e;
-  return launch_kernel(decode_split_kernel, dim3(a.d_c / 128, groups), dim3(C::THREADS), C::SMEM_BYTES, stream, pdl,
-                       map_ckv, map_krope, a);
+  return launch_kernel(kern, dim3(a.d_c / 128, groups), dim3(C::THREADS), C::SMEM_BYTES, stream, pdl, map_ckv,
+                       map_krope, a);
 }
 
 }  // namespace hra

@@ -335,6 +335,19 @@ __device__ __forceinline__ uint32_t bf16x2_to_f16x2(uint32_t v) {
   asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
   return r;
 }
+// Four int8 values (one 32-bit word, lowest byte first) times a scale -> four fp16 (two
+// packed words).  Each byte b is placed as the fp16 1024 + (b ^ 0x80) = 1152 + v (exact,
+// the spacing of fp16 in [1024, 2048) is 1), 1152 is subtracted (exact) and the integer
+// is multiplied by the scale (one fp16 rounding).
+__device__ __forceinline__ uint2 i8x4_to_f16x4(uint32_t w, __half2 scale) {
+  const uint32_t t = w ^ 0x80808080u;
+  const uint32_t lo = __byte_perm(t, 0x64646464u, 0x4140);  // bytes 0, 1 under 0x64 high bytes
+  const uint32_t hi = __byte_perm(t, 0x64646464u, 0x4342);  // bytes 2, 3
+  const __half2 bias = __float2half2_rn(1152.f);
+  __half2 a = __hmul2(__hsub2(*reinterpret_cast<const __half2*>(&lo), bias), scale);
+  __half2 b = __hmul2(__hsub2(*reinterpret_cast<const __half2*>(&hi), bias), scale);
+  return make_uint2(*reinterpret_cast<uint32_t*>(&a), *reinterpret_cast<uint32_t*>(&b));
+}
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   uint32_t r;
   asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));

@@ -64,7 +64,7 @@ typedef enum {
   HRA_ERR_DEVICE_TIMEOUT = -5   /* a bounded device-side wait expired                    */
 } hra_status;
 
-typedef enum { HRA_BF16 = 0, HRA_F32 = 1 } hra_dtype;
+typedef enum { HRA_BF16 = 0, HRA_F32 = 1, HRA_INT8 = 2 } hra_dtype;
 
 /*
  * Parameters of one decode step.  All pointers are device pointers, 16-byte aligned.
@@ -133,6 +133,21 @@ typedef struct {
   int out_accumulate;   /* 0 or 1                                                        */
   int n_out_peers;      /* 0..7 entries in out_peers (requires out_accumulate = 1)        */
   void* const* out_peers; /* host array of device pointers to [B, h, d_v] fp32, 16-B aligned */
+
+  /* Quantised latent cache (optional; 0 = the bf16 cache above).  The MLA tutorial's
+     deployment notes ("从MHA到MLA", 部署注意事项) serve MLA in INT8, and "Multi-Head
+     Low-Rank Attention" (未来方向) names KV-cache quantisation as the next step to combine
+     with MLRA.  cache_dtype = HRA_INT8: ckv holds int8 latent rows (ckv_stride counted in
+     bytes, a multiple of 16), each 128-column block b of row r standing for
+     q[r, c] * ckv_scale[r * ckv_scale_stride + b] (symmetric, one fp32 scale per token and
+     128-column block, i.e. per MLRA-4 branch; the caller writes both when it appends to the
+     cache).  krope stays bf16.  Supported for 128-wide branches (MLRA-4 and its branch
+     shards; others return HRA_ERR_UNSUPPORTED).  The decode kernel rescales each block
+     to fp16 (|q * scale| < 65504).  The cache then holds d_c + 2 * d_rope + 4 * d_c / 128
+     bytes per token instead of 2 * (d_c + d_rope).                                         */
+  hra_dtype cache_dtype;        /* HRA_BF16 (default) or HRA_INT8                          */
+  const float* ckv_scale;       /* fp32 scales, row r's at ckv_scale + r * ckv_scale_stride */
+  int64_t ckv_scale_stride;     /* floats between consecutive rows' scales, >= d_c / 128   */
 } hra_decode_params;
 
 /* Bytes of workspace one call with these parameters needs (0 on invalid parameters).
@@ -153,11 +168,14 @@ HRA_API hra_status mla_decode(const hra_decode_params* p, void* stream /* cudaSt
  * this is a deployment variant of mlra_decode.  Scratch comes from one 32 MiB
  * file-scope device array that every GPU loading the library holds until exit;
  * p->workspace and p->workspace_bytes are ignored.  Calls whose hra_workspace_size
- * exceeds 32 MiB return HRA_ERR_WORKSPACE before any CUDA call.  The first call on a
- * device looks the array's device address up (make it before any stream capture).
- * All calls on a device share the array: calls that overlap on the GPU race; the
- * status word is cleared by every call, and expired device waits recorded there are
- * not reachable through hra_check_device_status.  Allocates nothing. */
+ * exceeds 32 MiB return HRA_ERR_WORKSPACE before any launch (the size depends on batch,
+ * heads and the split count: with d_c = 512 and 37 splits, up to 35 sequences at h = 128
+ * and 74 at h = 16; the size check itself queries the current device's SM count unless
+ * num_splits > 0).  The first call on a device looks the array's device address up (make
+ * it before any stream capture); the address is kept, so do not use the library across a
+ * device reset.  All calls on a device share the array: calls that overlap on the GPU
+ * race; the status word is cleared by every call, and expired device waits recorded there
+ * are not reachable through hra_check_device_status.  Allocates nothing. */
 HRA_API hra_status mlra_decode_static(const hra_decode_params* p, void* stream /* cudaStream_t */);
 
 /* Synchronize `stream` and read the device status word of p->workspace.

@@ -311,6 +311,42 @@ def mlra_nope_key_blocks(c_kv, w_uk_i, n_blocks: int) -> np.ndarray:
     return sum(c_kv[:, b * w:(b + 1) * w] @ w_uk_i[b * w:(b + 1) * w] for b in range(n_blocks))
 
 
+def dequantize_int8_blocks(q, scale, block: int = 128) -> np.ndarray:
+    """The value an int8 latent cache stands for: x[r, c] = q[r, c] * scale[r, c // block].
+
+    Quantised latent cache ("从MHA到MLA", 部署注意事项: INT8 for inference; "Multi-Head
+    Low-Rank Attention", 未来方向: combine MLRA with KV-cache quantisation).  The pages fix
+    neither the scheme nor its granularity; read here as symmetric int8 with one scale per
+    token and 128-column latent block (one per MLRA-4 branch).  Exact in float64.
+    """
+    q = _f64(q)
+    s = _f64(scale)
+    rows, d = q.shape
+    return q * np.repeat(s[:, :d // block], block, axis=1)
+
+
+def decode_batch_int8(inp, wl, q8, scale, heads=None, seqs=None) -> np.ndarray:
+    """The absorbed oracle over a batch whose latent cache is int8 (q8 [rows, d_c] and
+    scale [rows, d_c / 128], physical rows like inp.cache): each sequence's latent rows are
+    dequantised (:func:`dequantize_int8_blocks`) and K_RoPE taken from inp.cache as it is."""
+    from synth import D_C
+    seqs = range(int(inp.seq_lens.shape[0])) if seqs is None else seqs
+    res = []
+    for s in seqs:
+        L = int(inp.seq_lens[s])
+        if inp.block_table is None:
+            phys = np.arange(s * inp.seq_stride, s * inp.seq_stride + L)
+        else:
+            t = np.arange(L)
+            P = wl.page_size
+            phys = inp.block_table.numpy()[s, t // P].astype(np.int64) * P + t % P
+        c = dequantize_int8_blocks(q8[phys], scale[phys])
+        res.append(mlra_decode_absorbed(inp.q[s], c, inp.cache[phys][:, D_C:], inp.w_uk, inp.w_uv, wl.n_branch,
+                                        alpha_q=wl.alpha_q, alpha_kv=wl.alpha_kv, branch_scale=wl.sigma_o,
+                                        softmax_scale=wl.softmax_scale, rope_theta=wl.rope_theta, heads=heads))
+    return np.stack(res)
+
+
 def decode_batch(inp, wl, heads=None, seqs=None, form: str = "absorbed") -> np.ndarray:
     """Run the oracle over sequences of a synth.Inputs; returns [len(seqs), len(heads), d_v]."""
     from synth import logical_rows, D_C

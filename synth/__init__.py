@@ -240,6 +240,24 @@ def logical_rows(inp: Inputs, wl: Workload, s: int) -> torch.Tensor:
     return inp.cache[phys]
 
 
+def quantize_int8_blocks(latent: torch.Tensor, block: int = 128):
+    """An int8 copy of a latent cache, as a caller would write it: for every row and
+    128-column block, scale = max|x| / 127 (fp32) and q = round-to-nearest-even(x / scale)
+    (0 where the block is all zero).  Returns (q int8 [rows, d], scale fp32 [rows, d / block]).
+
+    This is the cache format, not decode arithmetic: the decode (and the oracle) only read
+    it back as q * scale."""
+    x = latent.to(torch.float32)
+    rows, d = x.shape
+    xb = x.view(rows, d // block, block)
+    amax = xb.abs().amax(dim=2)
+    scale = amax / 127.0
+    safe = torch.where(scale > 0, scale, torch.ones_like(scale))
+    q = torch.round(xb / safe[:, :, None]).clamp_(-127, 127)
+    q = torch.where(scale[:, :, None] > 0, q, torch.zeros_like(q))
+    return q.to(torch.int8).view(rows, d), scale.contiguous()
+
+
 def kv_bytes(lens) -> int:
     """Algorithmic KV-cache bytes one decode step reads: 576 bf16 per cached token."""
     return int(np.asarray(lens, dtype=np.int64).sum()) * ROW * 2

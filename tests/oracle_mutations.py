@@ -28,6 +28,10 @@ MUTATIONS = [
     ("gla_decode", "heads = slice(g * per, (g + 1) * per)", "heads = slice(0, per)", "every group on the first heads"),
     ("mlra_prefill_expanded", "np.arange(L)[None, :] <= pos[:, None]", "np.arange(L)[None, :] < pos[:, None]",
      "causal mask hides the query's own token"),
+    ("dequantize_int8_blocks", "np.repeat(s[:, :d // block], block, axis=1)", "np.tile(s[:, :d // block], (1, block))",
+     "int8 block scales on the wrong columns"),
+    ("dequantize_int8_blocks", "return q * np.repeat", "return q / np.repeat", "int8 scale divided instead of multiplied"),
+    ("decode_batch_int8", "astype(np.int64) * P + t % P", "astype(np.int64) * P", "int8 cache page offset dropped"),
     ("mlra_prefill_expanded", "rope_rotate(q[j, i, d_nope:], int(pos[j]), rope_theta)",
      "rope_rotate(q[j, i, d_nope:], L - 1, rope_theta)", "every query rotated to the last position"),
 ]

@@ -151,3 +151,49 @@ def test_mla_decode_requires_one_branch():
 
 def test_workspace_size_zero_on_invalid():
     assert hra.load_library().hra_workspace_size(ctypes.byref(_fake_params(n_branch=5))) == 0
+
+
+@pytest.mark.parametrize("over,status", [
+    (dict(cache_dtype=B.HRA_INT8, n_branch=1, ckv_scale=0x90000, ckv_scale_stride=4), B.HRA_ERR_UNSUPPORTED),
+    (dict(cache_dtype=B.HRA_INT8, ckv_scale=None, ckv_scale_stride=4), B.HRA_ERR_INVALID_ARG),
+    (dict(cache_dtype=B.HRA_INT8, ckv_scale=0x90002, ckv_scale_stride=4), B.HRA_ERR_INVALID_ARG),  # misaligned
+    (dict(cache_dtype=B.HRA_INT8, ckv_scale=0x90000, ckv_scale_stride=3), B.HRA_ERR_INVALID_ARG),
+    (dict(cache_dtype=B.HRA_INT8, ckv_scale=0x90000, ckv_scale_stride=4, ckv_stride=584), B.HRA_ERR_INVALID_ARG),
+    (dict(cache_dtype=5), B.HRA_ERR_INVALID_ARG),
+    (dict(cache_dtype=B.HRA_INT8, ckv_scale=0x90000, ckv_scale_stride=4), B.HRA_ERR_WORKSPACE),
+])
+def test_int8_cache_fields_are_validated(over, status):
+    """An int8 latent cache needs 128-wide branches, 4-byte aligned scales with a row stride
+    of at least d_c / 128, and a 16-byte multiple row stride; a well-formed one passes
+    validation (and stops at the missing workspace)."""
+    p = _fake_params(**over)
+    rc = hra.load_library().mlra_decode(ctypes.byref(p), None)
+    assert rc == status, hra.last_error()
+
+
+def test_make_params_selects_the_int8_cache():
+    import torch
+    q = torch.zeros(1, 4, 192, dtype=torch.bfloat16)
+    ckv = torch.zeros(64, 512, dtype=torch.int8)
+    krope = torch.zeros(64, 64, dtype=torch.bfloat16)
+    scale = torch.ones(64, 4)
+    w = torch.zeros(4, 512, 128, dtype=torch.bfloat16)
+    out = torch.zeros(1, 4, 128)
+    p = hra.make_params(q, ckv, krope, torch.zeros(1, dtype=torch.int32), w, w, out, n_branch=4, ckv_scale=scale)
+    assert p.cache_dtype == B.HRA_INT8 and p.ckv_scale == scale.data_ptr() and p.ckv_scale_stride == 4
+    assert p.ckv_stride == 512
+    with pytest.raises(ValueError):
+        hra.make_params(q, ckv, krope, torch.zeros(1, dtype=torch.int32), w, w, out, n_branch=4)
+
+
+def test_static_entry_refuses_calls_beyond_its_array():
+    """The allocation-free entry point's 32 MiB array holds up to 35 sequences at h = 128
+    with d_c = 512 and 37 splits: B = 36 is refused before any device call; B = 35 passes
+    the size check (and then needs a device, which this host does not have)."""
+    big = _fake_params(batch=36, num_heads=128)
+    assert hra.load_library().mlra_decode_static(ctypes.byref(big), None) == B.HRA_ERR_WORKSPACE
+    assert "static array" in hra.last_error()
+    fits = _fake_params(batch=35, num_heads=128)
+    assert hra.load_library().mlra_decode_static(ctypes.byref(fits), None) != B.HRA_ERR_WORKSPACE
+    bad = _fake_params(n_branch=3)
+    assert hra.load_library().mlra_decode_static(ctypes.byref(bad), None) == B.HRA_ERR_UNSUPPORTED

@@ -363,3 +363,45 @@ def test_oracle_snapshot():
     inp = synth.make_inputs(wl)
     got = oracle.decode_batch(inp, wl, heads=fx["heads"], seqs=[0], form="expanded")[0]
     np.testing.assert_allclose(got, np.array(fx["out"]), rtol=1e-12, atol=1e-12)
+
+
+# --- quantised (int8) latent cache --------------------------------------------------------
+
+def test_int8_dequantize_places_each_block_scale_on_its_columns():
+    """x[r, c] = q[r, c] * scale[r, c // 128]; distinct power-of-two scales per block make
+    any mix-up of blocks, or a division for the product, visible exactly."""
+    rng = np.random.default_rng(11)
+    q = rng.integers(-127, 128, size=(6, 512)).astype(np.int8)
+    scale = np.array([[2.0 ** (b - r) for b in range(4)] for r in range(6)], dtype=np.float32)
+    x = oracle.dequantize_int8_blocks(q, scale)
+    expect = q.astype(np.float64) * (2.0 ** (np.arange(512)[None, :] // 128 - np.arange(6)[:, None]))
+    assert np.array_equal(x, expect)
+
+
+def test_int8_round_trip_within_half_a_step():
+    """The cache format (synth) read back by the oracle: every value is within half a
+    quantisation step of the bf16 value it stands for (plus the fp32 rounding of x / scale,
+    at most 127 * 2^-24 steps), and each block's largest value maps to +-127."""
+    x = (torch.randn(40, 512) * torch.tensor([0.5, 1.0, 4.0, 16.0]).repeat_interleave(128)).to(torch.bfloat16)
+    q, s = synth.quantize_int8_blocks(x)
+    back = oracle.dequantize_int8_blocks(q, s)
+    step = np.repeat(s.double().numpy(), 128, axis=1)
+    assert (np.abs(back - x.double().numpy()) <= (0.5 + 1e-4) * step).all()
+    assert (q.view(40, 4, 128).abs().amax(dim=2) == 127).all()
+
+
+@pytest.mark.parametrize("page_size", [0, 32])
+def test_int8_decode_on_integer_cache_equals_bf16_decode(page_size):
+    """Integer latent values in [-127, 127] with a 127 in every block quantise with scale
+    exactly 1, so the int8 decode must equal the bf16 decode of the same values."""
+    wl = synth.Workload("int8_pin", 4, 2, 4, 100, lengths=(37, 100), page_size=page_size)
+    inp = synth.make_inputs(wl)
+    rng = np.random.default_rng(5)
+    lat = rng.integers(-127, 128, size=(inp.cache.shape[0], 512)).astype(np.float32)
+    lat[:, ::128] = 127.0
+    inp.cache[:, :512] = torch.from_numpy(lat).to(torch.bfloat16)
+    q8, s = synth.quantize_int8_blocks(inp.cache[:, :512])
+    assert (s == 1.0).all()
+    got = oracle.decode_batch_int8(inp, wl, q8.numpy(), s.numpy())
+    ref = oracle.decode_batch(inp, wl)
+    assert _rel(got, ref) < 1e-12
