@@ -26,7 +26,8 @@ STATUS_NAMES = {0: "HRA_OK", -1: "HRA_ERR_INVALID_ARG", -2: "HRA_ERR_UNSUPPORTED
 
 # Symbols declared in include/hra.h.
 EXPORTS = ("hra_workspace_size", "mlra_decode", "mla_decode", "mlra_decode_static", "hra_check_device_status",
-           "hra_selftest_wait_timeout", "hra_last_error", "hra_version")
+           "hra_selftest_wait_timeout", "hra_last_error", "hra_version", "hra_prefill_workspace_size", "mlra_prefill",
+           "hra_check_prefill_status")
 
 
 class HraError(RuntimeError):
@@ -56,6 +57,23 @@ class HraDecodeParams(ctypes.Structure):
     ]
 
 
+class HraPrefillParams(ctypes.Structure):
+    """Mirror of hra_prefill_params (field order and C types as in include/hra.h)."""
+    _fields_ = [
+        ("num_heads", ctypes.c_int), ("n_branch", ctypes.c_int),
+        ("d_c", ctypes.c_int), ("d_rope", ctypes.c_int), ("d_nope", ctypes.c_int), ("d_v", ctypes.c_int),
+        ("seq_len", ctypes.c_int), ("n_query", ctypes.c_int),
+        ("q", ctypes.c_void_p), ("ckv", ctypes.c_void_p), ("krope", ctypes.c_void_p),
+        ("ckv_stride", ctypes.c_int64), ("krope_stride", ctypes.c_int64),
+        ("w_uk", ctypes.c_void_p), ("w_uv", ctypes.c_void_p),
+        ("alpha_q", ctypes.c_float), ("alpha_kv", ctypes.c_float), ("branch_scale", ctypes.c_float),
+        ("softmax_scale", ctypes.c_float), ("rope_theta", ctypes.c_float),
+        ("out", ctypes.c_void_p), ("out_dtype", ctypes.c_int),
+        ("workspace", ctypes.c_void_p), ("workspace_bytes", ctypes.c_size_t),
+        ("wait_limit", ctypes.c_int),
+    ]
+
+
 _lib: Optional[ctypes.CDLL] = None
 
 
@@ -72,6 +90,12 @@ def load_library() -> ctypes.CDLL:
     lib.hra_workspace_size.restype = ctypes.c_size_t
     for name in ("mlra_decode", "mla_decode", "mlra_decode_static", "hra_check_device_status"):
         getattr(lib, name).argtypes = [P, ctypes.c_void_p]
+        getattr(lib, name).restype = ctypes.c_int
+    PP = ctypes.POINTER(HraPrefillParams)
+    lib.hra_prefill_workspace_size.argtypes = [PP]
+    lib.hra_prefill_workspace_size.restype = ctypes.c_size_t
+    for name in ("mlra_prefill", "hra_check_prefill_status"):
+        getattr(lib, name).argtypes = [PP, ctypes.c_void_p]
         getattr(lib, name).restype = ctypes.c_int
     lib.hra_selftest_wait_timeout.argtypes = [ctypes.c_void_p, ctypes.c_int, ctypes.c_void_p]
     lib.hra_selftest_wait_timeout.restype = ctypes.c_int
@@ -195,3 +219,51 @@ def alloc_workspace(p: HraDecodeParams, device=None):
     ws = ws[off:off + n]
     p.workspace, p.workspace_bytes = ws.data_ptr(), n
     return ws
+
+
+def make_prefill_params(q, ckv, krope, w_uk, w_uv, out, *, n_branch: int, alpha_q: float = 1.0,
+                        alpha_kv: float = 1.0, branch_scale: Optional[float] = None, softmax_scale: float = 0.0,
+                        rope_theta: float = 10000.0, wait_limit: int = 0) -> HraPrefillParams:
+    """Fill hra_prefill_params from torch tensors: q [n, h, 192] bf16, ckv / krope 2-D row
+    views of the sequence's L cached rows, out [n, h, 128] (bf16 or fp32)."""
+    import torch
+    p = HraPrefillParams()
+    p.num_heads, p.n_branch = int(q.shape[1]), int(n_branch)
+    p.d_c, p.d_rope, p.d_nope, p.d_v = int(ckv.shape[1]), int(krope.shape[1]), int(q.shape[2]) - int(krope.shape[1]), int(w_uv.shape[2])
+    p.seq_len, p.n_query = int(ckv.shape[0]), int(q.shape[0])
+    p.q, p.ckv, p.krope = _ptr(q), _ptr(ckv), _ptr(krope)
+    p.ckv_stride, p.krope_stride = int(ckv.stride(0)), int(krope.stride(0))
+    p.w_uk, p.w_uv = _ptr(w_uk), _ptr(w_uv)
+    p.alpha_q, p.alpha_kv = float(alpha_q), float(alpha_kv)
+    p.branch_scale = float(1.0 / math.sqrt(n_branch) if branch_scale is None else branch_scale)
+    p.softmax_scale, p.rope_theta = float(softmax_scale), float(rope_theta)
+    p.out = _ptr(out)
+    p.out_dtype = HRA_F32 if out is not None and out.dtype == torch.float32 else HRA_BF16
+    p.wait_limit = int(wait_limit)
+    return p
+
+
+def prefill_workspace_size(p: HraPrefillParams) -> int:
+    n = load_library().hra_prefill_workspace_size(ctypes.byref(p))
+    if n == 0:
+        raise HraError(HRA_ERR_INVALID_ARG, last_error())
+    return int(n)
+
+
+def alloc_prefill_workspace(p: HraPrefillParams, device=None):
+    """Allocate a prefill workspace with torch (256-byte aligned) and attach it to p."""
+    import torch
+    n = prefill_workspace_size(p)
+    ws = torch.empty(n + 256, dtype=torch.uint8, device=device or "cuda")
+    off = (-ws.data_ptr()) % 256
+    ws = ws[off:off + n]
+    p.workspace, p.workspace_bytes = ws.data_ptr(), n
+    return ws
+
+
+def mlra_prefill(p: HraPrefillParams, stream=None) -> None:
+    _check(load_library().mlra_prefill(ctypes.byref(p), ctypes.c_void_p(_stream_handle(stream))))
+
+
+def check_prefill_status(p: HraPrefillParams, stream=None) -> None:
+    _check(load_library().hra_check_prefill_status(ctypes.byref(p), ctypes.c_void_p(_stream_handle(stream))))

@@ -16,6 +16,7 @@
 #include "hra.h"
 #include "absorb_combine.h"
 #include "decode_sm100.h"
+#include "prefill_sm100.h"
 #include "schedule.cuh"
 #include "sm100.cuh"
 
@@ -311,6 +312,133 @@ hra_status run_decode(const hra_decode_params* p, cudaStream_t stream) {
   return HRA_OK;
 }
 
+// ---------------------------------------------------------------------------- prefill
+constexpr long long kMaxPrefillLen = 1 << 20;
+
+hra_status validate_prefill(const hra_prefill_params* p) {
+  if (p == nullptr) return fail(HRA_ERR_INVALID_ARG, "params is NULL");
+  if (p->d_c != 512 || p->d_rope != 64 || p->d_nope != 128 || p->d_v != 128)
+    return fail(HRA_ERR_UNSUPPORTED, "widths (d_c=%d, d_rope=%d, d_nope=%d, d_v=%d) must be 512/64/128/128", p->d_c,
+                p->d_rope, p->d_nope, p->d_v);
+  if (p->n_branch != 1 && p->n_branch != 2 && p->n_branch != 4)
+    return fail(HRA_ERR_UNSUPPORTED, "n_branch=%d (supported: 1, 2, 4)", p->n_branch);
+  if (p->num_heads < 1 || p->num_heads > 128)
+    return fail(HRA_ERR_UNSUPPORTED, "num_heads=%d (supported: 1..128)", p->num_heads);
+  if (p->seq_len < 1 || p->seq_len > kMaxPrefillLen)
+    return fail(HRA_ERR_UNSUPPORTED, "seq_len=%d (supported: 1..%lld)", p->seq_len, kMaxPrefillLen);
+  if (p->n_query < 1 || p->n_query > p->seq_len)
+    return fail(HRA_ERR_INVALID_ARG, "n_query=%d must be in [1, seq_len=%d]", p->n_query, p->seq_len);
+  const struct { const void* ptr; const char* name; } ptrs[] = {
+      {p->q, "q"}, {p->ckv, "ckv"}, {p->krope, "krope"}, {p->w_uk, "w_uk"}, {p->w_uv, "w_uv"}, {p->out, "out"}};
+  for (const auto& x : ptrs) {
+    if (x.ptr == nullptr) return fail(HRA_ERR_INVALID_ARG, "%s is NULL", x.name);
+    if (!aligned16(x.ptr)) return fail(HRA_ERR_INVALID_ARG, "%s is not 16-byte aligned", x.name);
+  }
+  if (p->ckv_stride < 512 || p->ckv_stride % 8 != 0)
+    return fail(HRA_ERR_INVALID_ARG, "ckv_stride=%lld must be >= 512 and a multiple of 8", (long long)p->ckv_stride);
+  if (p->krope_stride < 64 || p->krope_stride % 8 != 0)
+    return fail(HRA_ERR_INVALID_ARG, "krope_stride=%lld must be >= 64 and a multiple of 8",
+                (long long)p->krope_stride);
+  if (p->out_dtype != HRA_BF16 && p->out_dtype != HRA_F32)
+    return fail(HRA_ERR_INVALID_ARG, "out_dtype=%d", (int)p->out_dtype);
+  if (p->wait_limit < 0) return fail(HRA_ERR_INVALID_ARG, "wait_limit=%d must be >= 0", p->wait_limit);
+  if (!std::isfinite(p->alpha_q) || !std::isfinite(p->alpha_kv) || !std::isfinite(p->branch_scale) ||
+      !std::isfinite(p->softmax_scale) || !(p->rope_theta > 0.f) || !std::isfinite(p->rope_theta))
+    return fail(HRA_ERR_INVALID_ARG, "scales must be finite and rope_theta > 0");
+  return HRA_OK;
+}
+
+struct PrefillPlan {
+  int l_pad = 0;
+  size_t q16 = 0, kr16 = 0, k_exp = 0, v_exp = 0, total = 0;
+};
+
+PrefillPlan prefill_plan(const hra_prefill_params* p) {
+  PrefillPlan pl;
+  pl.l_pad = (p->seq_len + 127) / 128 * 128;
+  const size_t h = static_cast<size_t>(p->num_heads);
+  size_t off = 256;  // status word
+  pl.q16 = off;
+  off = round256(off + static_cast<size_t>(p->n_query) * h * 192 * 2);
+  pl.kr16 = off;
+  off = round256(off + static_cast<size_t>(pl.l_pad) * 64 * 2);
+  pl.k_exp = off;
+  off = round256(off + static_cast<size_t>(p->n_branch) * h * pl.l_pad * 128 * 2);
+  pl.v_exp = off;
+  off = round256(off + static_cast<size_t>(p->n_branch) * h * pl.l_pad * 128 * 2);
+  pl.total = off;
+  return pl;
+}
+
+hra_status run_prefill(const hra_prefill_params* p, cudaStream_t stream) {
+  hra_status st = validate_prefill(p);
+  if (st != HRA_OK) return st;
+  const PrefillPlan pl = prefill_plan(p);
+  if (p->workspace == nullptr) return fail(HRA_ERR_WORKSPACE, "workspace is NULL");
+  if ((reinterpret_cast<uintptr_t>(p->workspace) & 255u) != 0)
+    return fail(HRA_ERR_WORKSPACE, "workspace is not 256-byte aligned");
+  if (p->workspace_bytes < pl.total)
+    return fail(HRA_ERR_WORKSPACE, "workspace_bytes=%zu < required %zu", p->workspace_bytes, pl.total);
+  uint8_t* ws = static_cast<uint8_t*>(p->workspace);
+  const int h = p->num_heads, nb = p->n_branch, L = p->seq_len, n = p->n_query;
+  hra::PrefillArgs a{};
+  a.q = static_cast<const __nv_bfloat16*>(p->q);
+  a.krope = static_cast<const __nv_bfloat16*>(p->krope);
+  a.krope_stride = p->krope_stride;
+  a.q16 = reinterpret_cast<__half*>(ws + pl.q16);
+  a.kr16 = reinterpret_cast<__half*>(ws + pl.kr16);
+  a.k_exp = reinterpret_cast<__half*>(ws + pl.k_exp);
+  a.v_exp = reinterpret_cast<__half*>(ws + pl.v_exp);
+  a.out_f32 = p->out_dtype == HRA_F32 ? static_cast<float*>(p->out) : nullptr;
+  a.out_bf16 = p->out_dtype == HRA_BF16 ? static_cast<__nv_bfloat16*>(p->out) : nullptr;
+  a.status = reinterpret_cast<int*>(ws);
+  a.heads = h;
+  a.n_branch = nb;
+  a.seq_len = L;
+  a.n_query = n;
+  a.l_pad = pl.l_pad;
+  a.alpha_q = p->alpha_q;
+  a.alpha_kv = p->alpha_kv;
+  a.branch_scale = p->branch_scale;
+  const float tau = p->softmax_scale > 0.f ? p->softmax_scale : 1.0f / std::sqrt(192.0f);
+  a.scale_log2 = tau * 1.4426950408889634f;
+  a.rope_theta = p->rope_theta;
+  const uint64_t limit_us = p->wait_limit > 0 ? static_cast<uint64_t>(p->wait_limit) : kDefaultWaitLimitUs;
+  a.wait_limit_ns = 1000ull * (limit_us < kMinWaitLimitUs ? kMinWaitLimitUs : limit_us);
+
+  hra::PrefillMaps m;
+  if ((st = encode_map(&m.ckv, p->ckv, 512, L, p->ckv_stride, 128)) != HRA_OK) return st;
+  if ((st = encode_map(&m.wuk, p->w_uk, 128, static_cast<int64_t>(h) * 512, 128, 128)) != HRA_OK) return st;
+  if ((st = encode_map(&m.wuv, p->w_uv, 128, static_cast<int64_t>(h) * 512, 128, 128)) != HRA_OK) return st;
+  // fp16 workspace tensors: the copies move 16-bit elements, whatever their format
+  if ((st = encode_map(&m.q16, a.q16, static_cast<int64_t>(h) * 192, n, static_cast<int64_t>(h) * 192, 128)) != HRA_OK)
+    return st;
+  const int64_t kv_rows = static_cast<int64_t>(nb) * h * pl.l_pad;
+  if ((st = encode_map(&m.k, a.k_exp, 128, kv_rows, 128, 128)) != HRA_OK) return st;
+  if ((st = encode_map(&m.v, a.v_exp, 128, kv_rows, 128, 128)) != HRA_OK) return st;
+  if ((st = encode_map(&m.kr16, a.kr16, 64, pl.l_pad, 64, 128)) != HRA_OK) return st;
+
+  cudaError_t e = cudaMemsetAsync(a.status, 0, 4 * sizeof(int), stream);
+  if (e != cudaSuccess) return cuda_fail(e, "status clear");
+  e = hra::launch_prefill(m, a, stream);
+  if (e != cudaSuccess) return cuda_fail(e, "prefill launch");
+  g_last_error.clear();
+  return HRA_OK;
+}
+
+hra_status read_status(void* workspace, cudaStream_t stream) {
+  cudaError_t e = cudaStreamSynchronize(stream);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");
+  int st[4] = {0, 0, 0, 0};
+  e = cudaMemcpy(st, workspace, sizeof(st), cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return cuda_fail(e, "status read");
+  if (st[0] != 0)
+    return fail(HRA_ERR_DEVICE_TIMEOUT, "device wait expired (code %d, site %d, parity %d, block %d)", st[0], st[1],
+                st[2], st[3]);
+  g_last_error.clear();
+  return HRA_OK;
+}
+
 __global__ void wait_timeout_selftest_kernel(int* status, uint64_t limit_ns) {
   __shared__ uint64_t bar;
   __shared__ volatile int abort_flag;
@@ -366,16 +494,21 @@ hra_status mla_decode(const hra_decode_params* p, void* stream) {
 
 hra_status hra_check_device_status(const hra_decode_params* p, void* stream) {
   if (p == nullptr || p->workspace == nullptr) return fail(HRA_ERR_INVALID_ARG, "params or workspace is NULL");
-  cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
-  if (e != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");
-  int st[4] = {0, 0, 0, 0};
-  e = cudaMemcpy(st, p->workspace, sizeof(st), cudaMemcpyDeviceToHost);
-  if (e != cudaSuccess) return cuda_fail(e, "status read");
-  if (st[0] != 0)
-    return fail(HRA_ERR_DEVICE_TIMEOUT, "device wait expired (code %d, site %d, parity %d, block %d)", st[0], st[1],
-                st[2], st[3]);
-  g_last_error.clear();
-  return HRA_OK;
+  return read_status(p->workspace, static_cast<cudaStream_t>(stream));
+}
+
+size_t hra_prefill_workspace_size(const hra_prefill_params* p) {
+  if (validate_prefill(p) != HRA_OK) return 0;
+  return prefill_plan(p).total;
+}
+
+hra_status mlra_prefill(const hra_prefill_params* p, void* stream) {
+  return run_prefill(p, static_cast<cudaStream_t>(stream));
+}
+
+hra_status hra_check_prefill_status(const hra_prefill_params* p, void* stream) {
+  if (p == nullptr || p->workspace == nullptr) return fail(HRA_ERR_INVALID_ARG, "params or workspace is NULL");
+  return read_status(p->workspace, static_cast<cudaStream_t>(stream));
 }
 
 hra_status hra_selftest_wait_timeout(void* workspace, int limit_us, void* stream) {

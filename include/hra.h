@@ -178,6 +178,54 @@ HRA_API hra_status mla_decode(const hra_decode_params* p, void* stream /* cudaSt
  * are not reachable through hra_check_device_status.  Allocates nothing. */
 HRA_API hra_status mlra_decode_static(const hra_decode_params* p, void* stream /* cudaStream_t */);
 
+/*
+ * Prefill: causal multi-token MLRA for one sequence, in the expanded form ("vllbc02MLA":
+ * prefill is compute-bound and works with the per-head keys and values; generation is
+ * memory-bound and uses the absorbed form).  The cache holds seq_len tokens; the queries
+ * are the last n_query of them (query j at position seq_len - n_query + j sees the tokens
+ * t <= its position), each attending per branch as in "Multi-Head Low-Rank Attention"
+ * (核心方法), with the branch outputs summed and scaled as in mlra_decode.
+ * The call forms K_nope^(b),(i) = alpha_kv C^(b) W_UK^(b),(i) and V^(b),(i) =
+ * alpha_kv C^(b) W_UV^(b),(i) for every cached token in the workspace (fp16), then runs
+ * a causal attention over them on the tensor cores (fp16 operands, fp32 accumulation,
+ * fp32 softmax).  With n_query = 1 it computes the same output as mlra_decode of that
+ * sequence.
+ * Supported: d_c = 512, n_branch in {1, 2, 4}, d_rope = 64, d_nope = d_v = 128,
+ * 1 <= num_heads <= 128, 1 <= n_query <= seq_len <= 2^20.  Pointers 16-byte aligned;
+ * the caller owns every buffer; the library allocates nothing.
+ */
+typedef struct {
+  int num_heads, n_branch;
+  int d_c, d_rope, d_nope, d_v;   /* 512, 64, 128, 128                                    */
+  int seq_len;          /* L, cached tokens including the queries                         */
+  int n_query;          /* n, query tokens: the last n positions                          */
+  const void* q;        /* bf16 [n, h, d_nope + d_rope], dense; q_rope NOT rotated        */
+  const void* ckv;      /* bf16 latent rows 0..L-1 of the sequence, ckv_stride apart      */
+  const void* krope;    /* bf16 rotated rope-key rows 0..L-1, krope_stride apart          */
+  int64_t ckv_stride, krope_stride;  /* elements; multiples of 8                         */
+  const void* w_uk;     /* bf16 [h, d_c, d_nope]                                          */
+  const void* w_uv;     /* bf16 [h, d_c, d_v]                                             */
+  float alpha_q, alpha_kv, branch_scale, softmax_scale, rope_theta;  /* as in mlra_decode */
+  void* out;            /* [n, h, d_v] in out_dtype                                       */
+  hra_dtype out_dtype;  /* HRA_BF16 or HRA_F32                                            */
+  void* workspace;      /* at least hra_prefill_workspace_size(p) bytes, 256-byte aligned */
+  size_t workspace_bytes;
+  int wait_limit;       /* as in hra_decode_params                                        */
+} hra_prefill_params;
+
+/* Workspace bytes of one prefill call (0 on invalid parameters): the status word, the
+ * fp16 queries, the fp16 rope keys and the expanded keys and values,
+ * 2 * n_branch * h * ceil(L / 128) * 128 * 128 fp16 values. */
+HRA_API size_t hra_prefill_workspace_size(const hra_prefill_params* p);
+
+/* Prefill (see above); asynchronous on `stream`.  Device-side expired waits are read back
+ * with hra_check_prefill_status. */
+HRA_API hra_status mlra_prefill(const hra_prefill_params* p, void* stream /* cudaStream_t */);
+
+/* Synchronize `stream` and read the device status word of p->workspace (as
+ * hra_check_device_status does for a decode call). */
+HRA_API hra_status hra_check_prefill_status(const hra_prefill_params* p, void* stream);
+
 /* Synchronize `stream` and read the device status word of p->workspace.
  * HRA_OK, or HRA_ERR_DEVICE_TIMEOUT if a bounded wait expired during the last call. */
 HRA_API hra_status hra_check_device_status(const hra_decode_params* p, void* stream);

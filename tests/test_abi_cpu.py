@@ -32,21 +32,23 @@ def test_library_loads_and_exports_every_declared_symbol():
     assert "sm_100a" in hra.version()
 
 
-def test_params_layout_matches_c(tmp_path):
-    fields = [f[0] for f in B.HraDecodeParams._fields_]
+@pytest.mark.parametrize("cls,ctype", [(B.HraDecodeParams, "hra_decode_params"),
+                                       (B.HraPrefillParams, "hra_prefill_params")])
+def test_params_layout_matches_c(tmp_path, cls, ctype):
+    fields = [f[0] for f in cls._fields_]
     prog = tmp_path / "layout.c"
     lines = ['#include <stdio.h>', '#include <stddef.h>', '#include "hra.h"', 'int main(void) {',
-             '  printf("size %zu\\n", sizeof(hra_decode_params));']
-    lines += [f'  printf("{f} %zu\\n", offsetof(hra_decode_params, {f}));' for f in fields]
+             f'  printf("size %zu\\n", sizeof({ctype}));']
+    lines += [f'  printf("{f} %zu\\n", offsetof({ctype}, {f}));' for f in fields]
     lines += ['  return 0;', '}']
     prog.write_text("\n".join(lines))
     exe = tmp_path / "layout"
     subprocess.run(["gcc", "-std=c99", f"-I{ROOT / 'include'}", str(prog), "-o", str(exe)], check=True)
     out = dict(line.split() for line in subprocess.run([str(exe)], capture_output=True, text=True,
                                                         check=True).stdout.splitlines())
-    assert int(out["size"]) == ctypes.sizeof(B.HraDecodeParams)
+    assert int(out["size"]) == ctypes.sizeof(cls)
     for f in fields:
-        assert int(out[f]) == getattr(B.HraDecodeParams, f).offset, f
+        assert int(out[f]) == getattr(cls, f).offset, f
 
 
 def _fake_params(**over):
@@ -197,3 +199,53 @@ def test_static_entry_refuses_calls_beyond_its_array():
     assert hra.load_library().mlra_decode_static(ctypes.byref(fits), None) != B.HRA_ERR_WORKSPACE
     bad = _fake_params(n_branch=3)
     assert hra.load_library().mlra_decode_static(ctypes.byref(bad), None) == B.HRA_ERR_UNSUPPORTED
+
+
+
+def _fake_prefill(**over):
+    """Well-formed prefill parameters with fake (aligned, never dereferenced) pointers."""
+    p = B.HraPrefillParams()
+    p.num_heads, p.n_branch = 16, 4
+    p.d_c, p.d_rope, p.d_nope, p.d_v = 512, 64, 128, 128
+    p.seq_len, p.n_query = 1000, 37
+    p.q, p.ckv, p.krope, p.w_uk, p.w_uv, p.out = 0x10000, 0x20000, 0x20400, 0x40000, 0x50000, 0x60000
+    p.ckv_stride, p.krope_stride = 576, 576
+    p.alpha_q = p.alpha_kv = 1.0
+    p.branch_scale, p.softmax_scale, p.rope_theta = 0.5, 0.0, 10000.0
+    p.out_dtype = B.HRA_F32
+    for k, v in over.items():
+        setattr(p, k, v)
+    return p
+
+
+@pytest.mark.parametrize("over,status", [
+    (dict(n_query=0), B.HRA_ERR_INVALID_ARG),
+    (dict(n_query=1001), B.HRA_ERR_INVALID_ARG),          # more queries than cached tokens
+    (dict(seq_len=0, n_query=0), B.HRA_ERR_UNSUPPORTED),
+    (dict(n_branch=3), B.HRA_ERR_UNSUPPORTED),
+    (dict(d_c=256), B.HRA_ERR_UNSUPPORTED),
+    (dict(num_heads=129), B.HRA_ERR_UNSUPPORTED),
+    (dict(q=0), B.HRA_ERR_INVALID_ARG),
+    (dict(ckv=0x20008), B.HRA_ERR_INVALID_ARG),           # misaligned
+    (dict(ckv_stride=500), B.HRA_ERR_INVALID_ARG),
+    (dict(out_dtype=7), B.HRA_ERR_INVALID_ARG),
+    (dict(), B.HRA_ERR_WORKSPACE),                        # well formed: stops at the missing workspace
+    (dict(workspace=0x80010, workspace_bytes=1 << 40), B.HRA_ERR_WORKSPACE),  # not 256-aligned
+])
+def test_prefill_validation_rejects_before_launch(over, status):
+    p = _fake_prefill(**over)
+    rc = hra.load_library().mlra_prefill(ctypes.byref(p), None)
+    assert rc == status, hra.last_error()
+
+
+def test_prefill_workspace_size_formula():
+    p = _fake_prefill()
+    r = lambda x: -(-x // 256) * 256
+    l_pad = 1024
+    expect = 256
+    expect = r(expect + 37 * 16 * 192 * 2)
+    expect = r(expect + l_pad * 64 * 2)
+    expect = r(expect + 4 * 16 * l_pad * 128 * 2)
+    expect = r(expect + 4 * 16 * l_pad * 128 * 2)
+    assert hra.prefill_workspace_size(p) == expect
+    assert hra.load_library().hra_prefill_workspace_size(ctypes.byref(_fake_prefill(n_branch=5))) == 0
