@@ -23,6 +23,10 @@ token.
 with half of the heads each (2.5 d_h of cache per token and rank); with one GPU, rank 0's
 call is timed alone, with 2 GPUs the ranks' outs are gathered over heads.
 
+--prefill L [--prefill-queries n]: the prefill path instead (causal multi-token MLRA-4 in the
+expanded form, h = 128, one sequence of L cached tokens whose last n are the queries), in
+TFLOP/s of algorithmic work against the measured tensor peak.
+
 --tp W (W = 2 or 4 for MLRA-4, 2 for MLRA-2): tensor parallelism by branch.  Rank r holds
 its W-th of the branches (cache columns + K_RoPE, W_UK / W_UV rows) and a step is its
 shard's decode followed by an NCCL all-reduce of out; run it with --gpus W.  With one GPU,
@@ -589,6 +593,112 @@ def run_native(args, wl, world, rank, local):
     del ws
 
 
+def prefill_flops(L: int, n: int, heads: int, n_branch: int = 4) -> int:
+    """Algorithmic FLOPs of one expanded-form prefill: forming K_nope and V for every cached
+    token (2 products of L x 512 x 128 per head) and, per head and branch, a 192-wide score
+    and a 128-wide P.V for every (query, visible key) pair."""
+    pairs = n * (L - n) + n * (n + 1) // 2
+    return 4 * L * 512 * 128 * heads + 2 * (192 + 128) * pairs * heads * n_branch
+
+
+def run_prefill_bench(args, world, rank, local):
+    """Prefill of one MLRA-4 sequence (h = 128): the three kernels of mlra_prefill per step."""
+    import head_rank_attention_b200 as hra
+    torch.cuda.set_device(local)
+    L = args.prefill
+    n = args.prefill_queries or L
+    wl = synth.Workload(f"prefill_mlra4_h128_L{L}_n{n}", 4, 1, 128, L)
+    inp = synth.make_inputs(wl)
+    q = synth.queries(synth.Workload(wl.name + "_q", 4, n, 128, L, seed=7))
+    dev = synth.to_device(inp)
+    cache = dev.cache[:L]
+    qd = q.cuda()
+    out = torch.empty(n, wl.heads, synth.D_V, dtype=torch.float32, device="cuda")
+    p = hra.make_prefill_params(qd, cache[:, :512], cache[:, 512:], dev.w_uk, dev.w_uv, out, n_branch=4,
+                                branch_scale=wl.sigma_o, softmax_scale=wl.softmax_scale, rope_theta=wl.rope_theta)
+    ws = hra.alloc_prefill_workspace(p)
+    stream = torch.cuda.current_stream()
+    for _ in range(args.warmup):
+        hra.mlra_prefill(p, stream)
+    hra.check_prefill_status(p, stream)
+    # the expanded keys and values (2 * 4 * 128 * L_pad * 128 fp16) exceed L2 from L = 512 on;
+    # below that, L2 is flushed before every step
+    flush = torch.zeros(128 << 20, dtype=torch.float32, device="cuda") if L < 1024 else None
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    pairs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    with ClockSampler(torch.cuda.current_device()) as clk:
+        for e0, e1 in pairs:
+            if flush is not None:
+                flush.add_(1)
+            e0.record(stream)
+            hra.mlra_prefill(p, stream)
+            e1.record(stream)
+        torch.cuda.synchronize()
+    hra.check_prefill_status(p, stream)
+    step_ms = statistics.median(e0.elapsed_time(e1) for e0, e1 in pairs)
+    # end to end: host copies of the query, the sequence's cache rows and the weights in, out back
+    pin = dict(q=q.pin_memory(), cache=inp.cache[:L].contiguous().pin_memory(), w_uk=inp.w_uk.pin_memory(),
+               w_uv=inp.w_uv.pin_memory())
+    dmap = dict(q=qd, cache=cache, w_uk=dev.w_uk, w_uv=dev.w_uv)
+    host_out = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
+    h2d = sum(t.numel() * t.element_size() for t in pin.values())
+    d2h = host_out.numel() * host_out.element_size()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    e2e_steps = max(1, min(args.steps, args.e2e_steps))
+    for _ in range(e2e_steps):
+        for k, t in pin.items():
+            dmap[k].copy_(t, non_blocking=True)
+        hra.mlra_prefill(p, stream)
+        host_out.copy_(out, non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1) / e2e_steps
+    step_ms, e2e_ms = max_over_ranks([step_ms, e2e_ms], world, "cuda")
+    if rank != 0:
+        return
+    flops = prefill_flops(L, n, wl.heads)
+    pk, pk_src = peaks()
+    tflops = world * flops / (step_ms * 1e-3) / 1e12
+    line = {
+        "metric": "MLRA-4 prefill TFLOP/s (expanded form)", "value": tflops, "unit": "TFLOP/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": step_ms, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f16",
+        "precision": "bf16 inputs; fp16 tensor-core operands (queries, expanded K/V); fp32 accumulate and softmax",
+        "data": "synthetic",
+        "config": {"workload": wl.name, "variant": "MLRA-4 prefill", "heads": wl.heads, "seq_len": L,
+                   "queries": n, "d_c": 512, "d_rope": 64, "flops_per_step": flops,
+                   "l2": "expanded K/V larger than L2; no flush" if flush is None else "512 MB written before every step"},
+        "roofline": {"bound": "tensor", "achieved": tflops / world, "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
+                     "frac": tflops / world / pk["bf16_tflops"], "peak_source": pk_src, "traffic": None,
+                     "note": "algorithmic FLOPs of the whole call (expansion + causal attention) over the "
+                             "measured dense bf16 peak (fp16 runs at the same rate)"},
+        "clocks": clk.summary(),
+        "e2e": {"value": world * flops / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s", "ms_per_step": e2e_ms,
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": e2e_steps},
+        "gpu_launches": 3 * args.steps,  # prep, expand, attend per step
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        # the oracle on a bounded sample (2 heads, the last min(n, 32) queries), scaled by FLOPs
+        hs, ns = 2, min(n, 32)
+        rows = inp.cache[:L]
+        t0 = time.perf_counter()
+        oracle_mod = __import__("oracle")
+        oracle_mod.mlra_prefill_expanded(q[n - ns:, :hs], rows[:, :512], rows[:, 512:], inp.w_uk[:hs], inp.w_uv[:hs], 4,
+                                         branch_scale=wl.sigma_o, softmax_scale=wl.softmax_scale,
+                                         rope_theta=wl.rope_theta)
+        dt = time.perf_counter() - t0
+        sample_flops = prefill_flops(L, ns, hs)
+        cpu_tflops = sample_flops / dt / 1e12
+        line["cpu_baseline"] = {"value": cpu_tflops, "unit": "TFLOP/s", "cores": os.cpu_count(), "kind": "oracle",
+                                "seconds_measured": dt,
+                                "sample": f"fp64 expanded prefill oracle on {hs} heads x the last {ns} queries "
+                                          f"(its own algorithmic FLOPs over its time)"}
+    print(json.dumps(line), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
@@ -612,6 +722,8 @@ def main():
                     help="latent cache format (int8: MLRA-4 workloads and their branch shards)")
     ap.add_argument("--gla", type=int, default=0, choices=[0, 2],
                     help="a rank of GLA-2 on an MLA workload (2 latent groups, half the heads each)")
+    ap.add_argument("--prefill", type=int, default=0, help="time the prefill path over this many cached tokens")
+    ap.add_argument("--prefill-queries", type=int, default=0, help="query tokens of --prefill (default: all)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -635,7 +747,13 @@ def main():
         ap.error(f"--gla {args.gla} runs on {args.gla} ranks (or one GPU for a single group), not {world}")
     if args.tp and world not in (1, args.tp):
         ap.error(f"--tp {args.tp} runs on {args.tp} ranks (or one GPU for a single shard), not {world}")
-    if args.impl == "reference":
+    if args.prefill:
+        if args.impl == "reference":
+            print(json.dumps({"impl": "reference", "unavailable": "the prefill mode has no reference arm; the oracle "
+                                                                  "sample is reported as cpu_baseline"}))
+            return
+        run_prefill_bench(args, world, rank, local)
+    elif args.impl == "reference":
         run_reference(args, wl, world, rank)
     else:
         run_native(args, wl, world, rank, local)

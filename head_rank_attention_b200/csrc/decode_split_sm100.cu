@@ -484,19 +484,24 @@ decode_split_kernel(const __grid_constant__ CUtensorMap map_ckv, const __grid_co
         uint32_t sr[HALF];
         tmem_load<HALF>(s_cols, sr);
         tmem_ld_wait();
-        float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-        if (n_mine == HALF) {
+        if (n_mine < HALF) {
 #pragma unroll
-          for (int k = 0; k < HALF; ++k) mx[k & 3] = fmaxf(mx[k & 3], __uint_as_float(sr[k]));
-        } else {
-#pragma unroll
-          for (int k = 0; k < HALF; ++k) {
+          for (int k = 0; k < HALF; ++k)
             if (k >= n_mine) sr[k] = __float_as_uint(-INFINITY);
-            mx[k & 3] = fmaxf(mx[k & 3], __uint_as_float(sr[k]));
-          }
         }
+        float mx[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) mx[q] = __uint_as_float(sr[q]);
+#pragma unroll
+        for (int k = 4; k + 8 <= HALF; k += 8)
+#pragma unroll
+          for (int q = 0; q < 4; ++q) mx[q] = fmax3(mx[q], __uint_as_float(sr[k + q]), __uint_as_float(sr[k + 4 + q]));
         const int rb = it & 1;
-        red_max[(rb * 2 + half) * 128 + row] = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
+        float mt4 = fmaxf(mx[0], mx[1]);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) mt4 = fmax3(mt4, mx[q], __uint_as_float(sr[HALF - 4 + q]));
+        red_max[(rb * 2 + half) * 128 + row] = mt4;
+
         warp_arrive(&red_bar[rb]);
         if (!warp_wait(&red_bar[rb], (it >> 1) & 1, limit, abort_flag, status, 33)) { ok = false; break; }
         const float mt = fmaxf(red_max[(rb * 2) * 128 + row], red_max[(rb * 2 + 1) * 128 + row]) * sl2;
@@ -509,16 +514,18 @@ decode_split_kernel(const __grid_constant__ CUtensorMap map_ckv, const __grid_co
           m_ref = mt;
           rescale = true;
         }
-        const float neg_m = -m_ref;
-        float sum[4] = {0.f, 0.f, 0.f, 0.f};
+        const float2 neg_m = make_float2(-m_ref, -m_ref);
+        const float2 sl2v = make_float2(sl2, sl2);
+        float2 s0 = make_float2(0.f, 0.f), s1 = make_float2(0.f, 0.f);
 #pragma unroll
         for (int k = 0; k < HALF / 2; ++k) {
-          const float p0 = ex2_approx(fmaf(__uint_as_float(sr[2 * k]), sl2, neg_m));
-          const float p1 = ex2_approx(fmaf(__uint_as_float(sr[2 * k + 1]), sl2, neg_m));
-          sum[k & 3] += p0 + p1;
-          sr[k] = pack_f16x2(p0, p1);
+          const float2 x = fma2(make_float2(__uint_as_float(sr[2 * k]), __uint_as_float(sr[2 * k + 1])), sl2v, neg_m);
+          const float2 pk = make_float2(ex2_approx(x.x), ex2_approx(x.y));
+          if (k & 1) s1 = add2(s1, pk); else s0 = add2(s0, pk);
+          sr[k] = pack_f16x2(pk.x, pk.y);
         }
-        const float tsum = (sum[0] + sum[1]) + (sum[2] + sum[3]);
+        const float2 st = add2(s0, s1);
+        const float tsum = st.x + st.y;
         l = first ? tsum : fmaf(l, factor, tsum);
         if (__any_sync(kAll, rescale)) {
           // every P.V so far must have completed before O is rescaled

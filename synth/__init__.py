@@ -115,6 +115,9 @@ WORKLOADS = {
     "paged_b64_t32k_mla": Workload("paged_b64_t32k_mla", 1, 64, 128, 32768, page_size=64),
     # MLRA-4 long context, B=4, lengths ~ U[65536, 131072]
     "long_mlra4_b4_t64k_128k": Workload("long_mlra4_b4_t64k_128k", 4, 4, 128, 131072, seq_len_min=65536),
+    # the paged MLRA-4 layout at 1/8 of the batch (302 MB of cache, still larger than L2): the
+    # size of a DRAM-traffic capture of the paged decode
+    "paged_b8_t32k_mlra4": Workload("paged_b8_t32k_mlra4", 4, 8, 128, 32768, page_size=64),
     # MLRA-4 very long context, B=1, T=2^21, 1% of positions with key norms x8
     "vlong_mlra4_b1_t2m": Workload("vlong_mlra4_b1_t2m", 4, 1, 128, 2097152, outlier_frac=0.01),
 }

@@ -149,3 +149,12 @@ def test_reference_arm_for_a_gla2_rank_reports_the_group():
     assert line["config"]["d_c"] == 256 and line["config"]["heads"] == 8
     assert line["config"]["variant"] == "GLA-2 rank"
     assert line["value"] == pytest.approx(2048 * (256 + 64) * 2 / (line["ms_per_step"] * 1e-3) / 1e12)
+
+
+def test_prefill_flop_count_matches_a_brute_count():
+    """The prefill bench's algorithmic FLOPs: K and V for every cached token, and per head and
+    branch a 192-wide score and a 128-wide P.V for every visible (query, key) pair."""
+    import bench
+    L, n, h, nb = 9, 4, 3, 4
+    pairs = sum(1 for j in range(n) for t in range(L) if t <= L - n + j)
+    assert bench.prefill_flops(L, n, h, nb) == 4 * L * 512 * 128 * h + 2 * 320 * pairs * h * nb
