@@ -522,7 +522,9 @@ def run_native(args, wl, world, rank, local):
         achieved_gbs = kv / (decode_ms * 1e-3) / 1e9
         flops = tensor_flops_per_token(n_branch, heads, d_c) * int(lens.astype(np.int64).sum())
         achieved_tflops = flops / (decode_ms * 1e-3) / 1e12
-        traffic = ncu_traffic(f"{wl.name}/tp{tpw}" if tpw else wl.name)
+        # recorded per workload, shard and cache format (the int8 cache is a different kernel)
+        traffic = ncu_traffic(wl.name + (f"/tp{tpw}" if tpw else "") + (f"/gla{gla}" if gla else "")
+                              + ("/int8" if int8 else ""))
         if gla:
             parallelism = (f"gla{gla}: head-and-latent groups, outs gathered over heads" if world == gla
                            else f"gla{gla}: rank 0's group alone (no gather)")
