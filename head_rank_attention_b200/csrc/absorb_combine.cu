@@ -25,6 +25,7 @@
 // output columns contiguous), streamed through two shared-memory stages in d_c / 128 K
 // chunks.  The branches partition the latent, so summing the per-branch up-projections
 // is this one contraction (and a branch shard's output is its part of that sum).
+#include <cooperative_groups.h>
 #include <cstdint>
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
@@ -202,6 +203,16 @@ absorb_tc_kernel(const __grid_constant__ CUtensorMap map_wuk, const __grid_const
   }
 }
 
+// Whether group g of G has a non-empty tile range over T tiles.  With T >= G every group
+// has one; otherwise (T < G <= 65535) the products below stay under 2^32, so the test needs
+// no 64-bit division.
+__device__ __forceinline__ bool group_live(int g, int G, int T) {
+  if (T >= G) return true;
+  const uint32_t t0 = static_cast<uint32_t>(g) * static_cast<uint32_t>(T) / static_cast<uint32_t>(G);
+  const uint32_t t1 = static_cast<uint32_t>(g + 1) * static_cast<uint32_t>(T) / static_cast<uint32_t>(G);
+  return t0 != t1;
+}
+
 // ---------------------------------------------------------------------------- merge
 // grid (ceil(h / (256 / TPH)), d_c / 128 slices, B), 256 * Z threads.  Thread = (head, CPT
 // consecutive latent columns of the slice); the Z thread sets take alternate runs of GU
@@ -234,7 +245,7 @@ __global__ void __launch_bounds__(256 * Z) merge_kernel(const CombineArgs a) {
       for (int u = 0; u < GU; ++u) {
         const int g = gb + u;
         // a group with an empty tile range (more groups than tiles) wrote nothing
-        const bool live = g <= g_hi && group_tile_begin(g, G, T) != group_tile_begin(g + 1, G, T);
+        const bool live = g <= g_hi && group_live(g, G, T);
         const long long row = ((static_cast<long long>(g) + seq) * gridDim.y + slice) * 128 + head;
         ml[u] = live ? a.ml_part[row] : make_float2(-INFINITY, 0.f);
 #pragma unroll
@@ -488,6 +499,188 @@ upproj_tc_kernel(const __grid_constant__ CUtensorMap map_wuv, const __grid_const
   }
 }
 
+// ---------------------------------------------------------------------------- small batches
+// Merge + up-projection in one kernel for B <= kSmallBatch, where the two kernels above are
+// bound by their load latencies (the merge's dependent rounds over many groups, the
+// up-projection's 128-row MMA tiles holding a few sequences).  Grid (d_c / 128 slices, h)
+// in clusters of the slices of one head, 512 threads.  CTA (slice c, head i):
+//   1. reads W_UV[i] rows [128 c, 128 c + 128) into registers (thread = 16 rows x 2
+//      columns) before waiting for the decode, since no kernel of the call writes it;
+//   2. merges the split partials of slice c for every sequence: the (sequence, group)
+//      pairs are laid end to end and thread set z = t / 128 takes every fourth one, all of
+//      its loads issued before any is used; the four sets are combined in shared memory;
+//   3. multiplies the merged latent row by its W_UV rows (fp32 sums) and leaves the partial
+//      output of each sequence in shared memory;
+//   4. cluster rank 0 adds the slices' partials (distributed shared memory) and writes out.
+// The only waits are the two cluster barriers, which every thread of every CTA reaches.
+constexpr int kSmallThreads = 512;
+constexpr int kSmallLoads = 10;  // (sequence, group) pairs a thread set loads per round
+
+__global__ void __launch_bounds__(kSmallThreads, 2) combine_small_kernel(const CombineArgs a) {
+  constexpr int SB = kSmallBatch;
+  namespace cg = cooperative_groups;
+  cg::cluster_group cluster = cg::this_cluster();
+  __shared__ float x_acc[4][SB][128];
+  __shared__ float2 x_md[4][SB][128];
+  __shared__ float o_lat[SB][128];
+  __shared__ float red[8][SB][128];
+  __shared__ float part[SB][128];
+  __shared__ int seg_pre[SB + 1], seg_gl[SB];
+  const int t = threadIdx.x;
+  const int c = blockIdx.x, slices = gridDim.x, i = blockIdx.y;
+  if (t == 0) grid_dep_launch();
+
+  // 1. W_UV rows 128 c + 16 rg + k (k < 16), columns 2 cp and 2 cp + 1
+  const int rg = t >> 6, cp = t & 63;
+  uint32_t w[16];
+  {
+    const uint32_t* src =
+        reinterpret_cast<const uint32_t*>(a.w_uv + (static_cast<long long>(i) * a.d_c + 128 * c + 16 * rg) * 128) + cp;
+#pragma unroll
+    for (int k = 0; k < 16; ++k) w[k] = __ldg(src + 64 * k);
+  }
+  grid_dep_wait();  // the split partials and the tile prefix come from the previous kernels
+
+  // 2. merge.  Lane s of warp 0 finds sequence s's group range [g_lo, g_lo + n); the ranges
+  // are laid end to end (pair q of sequence s is group gl[s] + q).
+  const int z = t >> 7, j = t & 127;
+  const int B = a.batch, G = a.groups, T = a.tile_prefix[B];
+  if (t < 32) {
+    int g0 = 0, n = 0;
+    if (t < B) {
+      const int p0 = a.tile_prefix[t], p1 = a.tile_prefix[t + 1];
+      if (p1 > p0) {
+        g0 = group_of_tile(p0, G, T);
+        n = group_of_tile(p1 - 1, G, T) - g0 + 1;
+      }
+    }
+    int incl = n;  // inclusive prefix over the (at most SB) sequences
+#pragma unroll
+    for (int off = 1; off < SB; off <<= 1) {
+      const int v = __shfl_up_sync(0xffffffffu, incl, off);
+      if (t >= off) incl += v;
+    }
+    if (t < SB) {
+      seg_pre[t + 1] = incl;
+      seg_gl[t] = g0 - (incl - n);
+    }
+    if (t == 0) seg_pre[0] = 0;
+  }
+  __syncthreads();
+  int gl[SB], pre[SB + 1];
+#pragma unroll
+  for (int s = 0; s <= SB; ++s) pre[s] = seg_pre[s];
+#pragma unroll
+  for (int s = 0; s < SB; ++s) gl[s] = seg_gl[s];
+  float acc[SB], M[SB], den[SB];
+#pragma unroll
+  for (int s = 0; s < SB; ++s) {
+    acc[s] = 0.f;
+    M[s] = -INFINITY;
+    den[s] = 0.f;
+  }
+  for (int q0 = z; q0 < pre[SB]; q0 += 4 * kSmallLoads) {
+    float2 ml[kSmallLoads];
+    float o[kSmallLoads];
+    int sq[kSmallLoads];
+#pragma unroll
+    for (int u = 0; u < kSmallLoads; ++u) {
+      const int q = q0 + 4 * u;
+      int s = 0;
+#pragma unroll
+      for (int k = 1; k < SB; ++k) s += q >= pre[k] ? 1 : 0;
+      int g = q;
+#pragma unroll
+      for (int k = 0; k < SB; ++k) g += s == k ? gl[k] : 0;
+      // a group with an empty tile range (more groups than tiles) wrote nothing
+      const bool live = q < pre[SB] && group_live(g, G, T);
+      const int row = ((g + s) * slices + c) * 128 + i;  // < (65535 + 1024) * 4 * 128
+      sq[u] = s;
+      ml[u] = live ? a.ml_part[row] : make_float2(-INFINITY, 0.f);
+      o[u] = live ? a.o_part[static_cast<long long>(row) * 128 + j] : 0.f;
+    }
+#pragma unroll
+    for (int u = 0; u < kSmallLoads; ++u) {
+      if (ml[u].x == -INFINITY) continue;
+#pragma unroll
+      for (int s = 0; s < SB; ++s) {
+        if (sq[u] != s) continue;
+        const float mx = fmaxf(M[s], ml[u].x);
+        const float r = ex2_approx(M[s] - mx), wt = ex2_approx(ml[u].x - mx);
+        den[s] = fmaf(den[s], r, wt * ml[u].y);
+        acc[s] = fmaf(acc[s], r, wt * o[u]);
+        M[s] = mx;
+      }
+    }
+  }
+#pragma unroll
+  for (int s = 0; s < SB; ++s) {
+    x_acc[z][s][j] = acc[s];
+    x_md[z][s][j] = make_float2(M[s], den[s]);
+  }
+  __syncthreads();
+  if (z < SB) {  // thread (sequence z, column j) combines the four sets
+    const int s = z;
+    float mx = -INFINITY;
+#pragma unroll
+    for (int k = 0; k < 4; ++k) mx = fmaxf(mx, x_md[k][s][j].x);
+    float num = 0.f, d = 0.f;
+    if (mx != -INFINITY) {
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const float2 md = x_md[k][s][j];
+        const float wt = ex2_approx(md.x - mx);
+        d = fmaf(wt, md.y, d);
+        num = fmaf(wt, x_acc[k][s][j], num);
+      }
+    }
+    o_lat[s][j] = d > 0.f ? num / d : 0.f;  // an empty sequence gives zeros
+  }
+  __syncthreads();
+
+  // 3. partial up-projection over this slice's 128 latent rows
+#pragma unroll
+  for (int s = 0; s < SB; ++s) {
+    if (s >= B) break;
+    float2 y = make_float2(0.f, 0.f);
+#pragma unroll
+    for (int k = 0; k < 16; ++k) {
+      const float x = o_lat[s][16 * rg + k];
+      const float2 wf = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w[k]));
+      y.x = fmaf(x, wf.x, y.x);
+      y.y = fmaf(x, wf.y, y.y);
+    }
+    red[rg][s][2 * cp] = y.x;
+    red[rg][s][2 * cp + 1] = y.y;
+  }
+  __syncthreads();
+  if (z < SB && z < B) {
+    float y = 0.f;
+#pragma unroll
+    for (int k = 0; k < 8; ++k) y += red[k][z][j];
+    part[z][j] = y;
+  }
+
+  // 4. rank 0 of the head's cluster sums the slices and writes out
+  cluster.sync();
+  if (cluster.block_rank() == 0 && z < SB && z < B) {
+    const int s = z;
+    float y = part[s][j];
+    for (int r = 1; r < slices; ++r) y += *cluster.map_shared_rank(&part[s][j], r);
+    y *= a.branch_scale * a.alpha_kv;
+    const long long o = (static_cast<long long>(s) * a.heads + i) * 128 + j;
+    if (a.out_f32 && a.accumulate) {
+      atomicAdd(a.out_f32 + o, y);
+      for (int k = 0; k < a.n_peers; ++k) atomicAdd(a.peers[k] + o, y);
+    } else if (a.out_f32) {
+      a.out_f32[o] = y;
+    } else {
+      a.out_bf16[o] = __float2bfloat16_rn(y);
+    }
+  }
+  cluster.sync();  // the other slices keep their shared memory until rank 0 has read it
+}
+
 template <class K>
 cudaError_t set_smem(K kern, int bytes) {
   return cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
@@ -509,6 +702,13 @@ cudaError_t launch_absorb_q(const CUtensorMap& map_wuk, const CUtensorMap& map_q
 
 cudaError_t launch_combine_upproj(const CUtensorMap& map_wuv, const CUtensorMap& map_olat, const CombineArgs& a,
                                   cudaStream_t stream, bool pdl) {
+  // The fused kernel takes one CTA per (head, slice) and one or two load rounds per thread
+  // set for up to 64 groups: used where that grid fits on the SMs at once.  With more heads
+  // or groups the merge kernel and the tensor-core up-projection are faster (measured at
+  // h = 128 with 37 and 148 groups).
+  if (a.batch <= kSmallBatch && (a.d_c / 128) * a.heads <= a.sms && a.groups <= 64)
+    return launch_kernel_cluster(combine_small_kernel, dim3(a.d_c / 128, a.heads), dim3(kSmallThreads), 0, stream, pdl,
+                                 a.d_c / 128, a);
   // Many sequences: 32 heads x 4 float4 per block.  Few sequences (each spread over many
   // groups): 8 heads x 1 float4 per block and two thread sets over alternate group runs.
   cudaError_t e;

@@ -28,6 +28,7 @@ struct CombineArgs {
   const float2* ml_part;      // [slots, d_c / 128, 128]
   const int* tile_prefix;     // [B + 1], written by the absorb kernel
   __nv_bfloat16* o_lat;       // merged latent output, bf16 hi [h, B, d_c] then bf16 lo [h, B, d_c]
+  const __nv_bfloat16* w_uv;  // [h, d_c, 128] (read directly by the small-batch combine)
   int* status;                // device status word (expired waits)
   float* out_f32;             // [B, h, 128] or nullptr
   __nv_bfloat16* out_bf16;    // [B, h, 128] or nullptr
@@ -36,6 +37,7 @@ struct CombineArgs {
   float* peers[kMaxOutPeers]; // other ranks' out buffers (peer memory), [B, h, 128] fp32
   int batch, heads, groups;
   int d_c;                    // latent width (as in AbsorbArgs)
+  int sms;                    // streaming multiprocessors of the device
   float alpha_kv, branch_scale;
 };
 
@@ -49,6 +51,9 @@ int upproj_seq_chunk();
 // pdl: launch with programmatic dependent launch (launch.h).
 cudaError_t launch_absorb_q(const CUtensorMap& map_wuk, const CUtensorMap& map_q, const AbsorbArgs& a,
                             cudaStream_t stream, bool pdl);
+// Batches of up to kSmallBatch sequences with few heads take one fused merge + up-projection
+// kernel; the others the merge kernel and the tensor-core up-projection.
+constexpr int kSmallBatch = 4;
 // map_wuv:  W_UV viewed as [h*d_c rows, 128] bf16, box {64, 128}, SWIZZLE_128B.
 // map_olat: a.o_lat viewed as [2*h*B rows, d_c] bf16, box {64, upproj_seq_chunk()}, SWIZZLE_128B.
 cudaError_t launch_combine_upproj(const CUtensorMap& map_wuv, const CUtensorMap& map_olat, const CombineArgs& a,

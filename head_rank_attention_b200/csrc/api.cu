@@ -293,6 +293,7 @@ hra_status run_decode(const hra_decode_params* p, cudaStream_t stream) {
   cb.ml_part = ml_part;
   cb.tile_prefix = tile_prefix;
   cb.o_lat = o_lat;
+  cb.w_uv = static_cast<const __nv_bfloat16*>(p->w_uv);
   cb.status = status;
   cb.out_f32 = p->out_dtype == HRA_F32 ? static_cast<float*>(p->out) : nullptr;
   cb.out_bf16 = p->out_dtype == HRA_BF16 ? static_cast<__nv_bfloat16*>(p->out) : nullptr;
@@ -303,6 +304,7 @@ hra_status run_decode(const hra_decode_params* p, cudaStream_t stream) {
   cb.heads = p->num_heads;
   cb.groups = plan.groups;
   cb.d_c = dc;
+  if ((st = sm_count(&cb.sms)) != HRA_OK) return st;
   cb.alpha_kv = p->alpha_kv;
   cb.branch_scale = p->branch_scale;
   e = hra::launch_combine_upproj(map_wuv, map_olat, cb, stream, pdl);
