@@ -228,9 +228,11 @@ hra_status run_decode(const hra_decode_params* p, cudaStream_t stream) {
     return st;
   const bool int8 = p->cache_dtype == HRA_INT8;
   // int8: one 128-byte box per 128-wide branch and 32 rows; bf16: 64-column boxes
-  if ((st = encode_map(&map_ckv, p->ckv, dc, p->cache_rows, p->ckv_stride, 32, int8, int8 ? 128 : 64)) != HRA_OK)
+  const int box_rows = int8 ? 32 : hra::decode_box_rows(dc / p->n_branch);
+  if ((st = encode_map(&map_ckv, p->ckv, dc, p->cache_rows, p->ckv_stride, box_rows, int8, int8 ? 128 : 64)) !=
+      HRA_OK)
     return st;
-  if ((st = encode_map(&map_krope, p->krope, 64, p->cache_rows, p->krope_stride, 32)) != HRA_OK) return st;
+  if ((st = encode_map(&map_krope, p->krope, 64, p->cache_rows, p->krope_stride, box_rows)) != HRA_OK) return st;
 
   auto mark = [&](int k) -> cudaError_t {
     return p->stage_events ? cudaEventRecord(static_cast<cudaEvent_t>(p->stage_events[k]), stream) : cudaSuccess;

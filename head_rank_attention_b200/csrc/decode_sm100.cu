@@ -49,7 +49,8 @@ struct DecodeCfg {
   static constexpr int SLICES_PER_BRANCH = W / 128;
   static constexpr int BOX_BYTES = NT * 128;         // one 64-column box over NT rows
   static constexpr int STAGE_BYTES = QK_BOXES * BOX_BYTES;
-  static constexpr int CHUNKS = NT / 32;             // TMA row chunks per tile
+  static constexpr int CHUNK_ROWS = NT % 32 == 0 ? 32 : 16;  // rows of one TMA box
+  static constexpr int CHUNKS = NT / CHUNK_ROWS;     // TMA row chunks per tile
   static constexpr int HALF = NT / 2;                // score columns per softmax thread
   static constexpr int TMEM_O = 0;                   // O: 128 fp32 columns
   static constexpr int TMEM_S = 128;                 // S/P double buffer: 2 x NT columns
@@ -62,7 +63,8 @@ struct DecodeCfg {
   static constexpr int MISC_BYTES = BAR_BYTES + RED_BYTES + 4 * (kMaxBatch + 1);
   static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + MISC_BYTES;
   static_assert(TMEM_Q + QK_DIMS / 2 <= TMEM_COLS, "TMEM budget");
-  static_assert(NT % 32 == 0 && NT >= 32 && NT <= 256, "tile rows");
+  static_assert(NT % 16 == 0 && NT >= 32 && NT <= 256, "tile rows");
+  static_assert(BOX_BYTES % 1024 == 0, "128-byte swizzle atoms");
   static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 };
 
@@ -174,7 +176,7 @@ decode_kernel(const __grid_constant__ CUtensorMap map_ckv, const __grid_constant
   if (warp == 12) {
     // ------------------------------------------------------------------ TMA producer
     // The CTA's tiles are the global tiles t_begin .. t_end-1 in order.  Each lane finds
-    // the cache row of one 32-row chunk of a batch of 32 / CHUNKS tiles (block-table and
+    // the cache row of one CHUNK_ROWS-row chunk of a batch of 32 / CHUNKS tiles (block-table and
     // length loads in parallel), one batch ahead of the tiles lane 0 is issuing, so that
     // no dependent global load sits between two tiles' copies.
     constexpr int TPB = 32 / C::CHUNKS;
@@ -184,7 +186,7 @@ decode_kernel(const __grid_constant__ CUtensorMap map_ckv, const __grid_constant
       const int t = t_begin + it0 + lane / C::CHUNKS;
       if (t >= t_end) return static_cast<int>(a.cache_rows);
       const int s = seq_of_tile(prefix, B, t);
-      return cache_chunk_row(a, s, (t - prefix[s]) * NT + 32 * (lane % C::CHUNKS));
+      return cache_chunk_row(a, s, (t - prefix[s]) * NT + C::CHUNK_ROWS * (lane % C::CHUNKS));
     };
     int rows = chunk_row(0);
     int issued = 0;
@@ -207,7 +209,7 @@ decode_kernel(const __grid_constant__ CUtensorMap map_ckv, const __grid_constant
           for (int r = 0; r < C::CHUNKS; ++r) {
 #pragma unroll
             for (int d = 0; d < C::QK_BOXES; ++d) {
-              void* box = dst + d * C::BOX_BYTES + r * 4096;
+              void* box = dst + d * C::BOX_BYTES + r * C::CHUNK_ROWS * 128;
               if (d < C::QK_BOXES - 1)
                 tma_load_2d(box, &map_ckv, &full[stage], branch * C::W + 64 * d, y[r], policy);
               else
@@ -493,8 +495,10 @@ cudaError_t launch_decode(const CUtensorMap& map_ckv, const CUtensorMap& map_kro
 }  // namespace
 
 int decode_tile_tokens(int branch_width) {
-  return branch_width == 128 ? decode_split_tile_tokens() : (branch_width == 256 ? 64 : 32);
+  return branch_width == 128 ? decode_split_tile_tokens() : (branch_width == 256 ? 64 : 48);
 }
+
+int decode_box_rows(int branch_width) { return branch_width == 512 ? DecodeCfg<1, 48, 4>::CHUNK_ROWS : 32; }
 
 cudaError_t launch_decode_kernel(int n_branch, const CUtensorMap& map_ckv, const CUtensorMap& map_krope,
                                  const DecodeArgs& a, int groups, cudaStream_t stream, bool pdl) {
@@ -502,7 +506,7 @@ cudaError_t launch_decode_kernel(int n_branch, const CUtensorMap& map_ckv, const
   switch (a.d_c / n_branch) {  // branch width
     case 128: return launch_decode_split_kernel(map_ckv, map_krope, a, groups, stream, pdl);
     case 256: return launch_decode<2, 64, 5>(map_ckv, map_krope, a, groups, stream, pdl);
-    case 512: return launch_decode<1, 32, 5>(map_ckv, map_krope, a, groups, stream, pdl);
+    case 512: return launch_decode<1, 48, 4>(map_ckv, map_krope, a, groups, stream, pdl);
     default: return cudaErrorInvalidValue;
   }
 }

@@ -57,9 +57,11 @@ __device__ __forceinline__ int cache_chunk_row(const DecodeArgs& a, int s, int t
 // Tokens per cache tile for a branch width (decides the TMEM and shared-memory budget).
 int decode_tile_tokens(int branch_width);
 int decode_split_tile_tokens();
+// Rows of one TMA box of the bf16 cache (the tensor maps' box height) for a branch width.
+int decode_box_rows(int branch_width);
 
-// 128-wide-branch kernel (MLRA-4, or a shard of its branches) on the bf16 cache with a
-// two-term bf16 query; grid (d_c / 128 branches, groups).
+// 128-wide-branch kernel (MLRA-4, or a shard of its branches) with an fp16 query and the
+// tile converted to fp16 in shared memory; grid (d_c / 128 branches, groups).
 cudaError_t launch_decode_split_kernel(const CUtensorMap& map_ckv, const CUtensorMap& map_krope,
                                        const DecodeArgs& a, int groups, cudaStream_t stream, bool pdl);
 

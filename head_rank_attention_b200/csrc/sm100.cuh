@@ -270,30 +270,48 @@ __device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t* r) {
                "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7])
                : "memory");
 }
-// N consecutive 32-bit TMEM columns of this warp's 32 lanes <-> registers (N a multiple of 16 / 8).
+__device__ __forceinline__ void tmem_ld8(uint32_t taddr, uint32_t* r) {
+  asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7])
+               : "r"(taddr));
+}
+__device__ __forceinline__ void tmem_st4(uint32_t taddr, const uint32_t* r) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x4.b32 [%0], {%1,%2,%3,%4};" ::"r"(taddr), "r"(r[0]), "r"(r[1]),
+               "r"(r[2]), "r"(r[3])
+               : "memory");
+}
+// N consecutive 32-bit TMEM columns of this warp's 32 lanes <-> registers, in pieces of
+// 32, 16, 8 (loads) or 4 (stores) columns: the widest width that divides N, so that every
+// piece starts at a column that is a multiple of its width whenever taddr is.
 template <int N>
 __device__ __forceinline__ void tmem_load(uint32_t taddr, uint32_t* r) {
-  static_assert(N % 16 == 0, "tmem_load width");
+  static_assert(N % 8 == 0, "tmem_load width");
   if constexpr (N % 32 == 0) {
 #pragma unroll
     for (int k = 0; k < N / 32; ++k) tmem_ld32(taddr + 32 * k, r + 32 * k);
-  } else {
+  } else if constexpr (N % 16 == 0) {
 #pragma unroll
     for (int k = 0; k < N / 16; ++k) tmem_ld16(taddr + 16 * k, r + 16 * k);
+  } else {
+#pragma unroll
+    for (int k = 0; k < N / 8; ++k) tmem_ld8(taddr + 8 * k, r + 8 * k);
   }
 }
 template <int N>
 __device__ __forceinline__ void tmem_store(uint32_t taddr, const uint32_t* r) {
-  static_assert(N % 8 == 0, "tmem_store width");
+  static_assert(N % 4 == 0, "tmem_store width");
   if constexpr (N % 32 == 0) {
 #pragma unroll
     for (int k = 0; k < N / 32; ++k) tmem_st32(taddr + 32 * k, r + 32 * k);
   } else if constexpr (N % 16 == 0) {
 #pragma unroll
     for (int k = 0; k < N / 16; ++k) tmem_st16(taddr + 16 * k, r + 16 * k);
-  } else {
+  } else if constexpr (N % 8 == 0) {
 #pragma unroll
     for (int k = 0; k < N / 8; ++k) tmem_st8(taddr + 8 * k, r + 8 * k);
+  } else {
+#pragma unroll
+    for (int k = 0; k < N / 4; ++k) tmem_st4(taddr + 4 * k, r + 4 * k);
   }
 }
 __device__ __forceinline__ void tmem_ld_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
