@@ -495,17 +495,20 @@ cudaError_t launch_decode(const CUtensorMap& map_ckv, const CUtensorMap& map_kro
 }  // namespace
 
 int decode_tile_tokens(int branch_width) {
-  return branch_width == 128 ? decode_split_tile_tokens() : (branch_width == 256 ? 64 : 48);
+  return branch_width == 128 ? decode_split_tile_tokens() : (branch_width == 256 ? 80 : 48);
 }
 
-int decode_box_rows(int branch_width) { return branch_width == 512 ? DecodeCfg<1, 48, 4>::CHUNK_ROWS : 32; }
+int decode_box_rows(int branch_width) {
+  return branch_width == 512 ? DecodeCfg<1, 48, 4>::CHUNK_ROWS
+                             : (branch_width == 256 ? DecodeCfg<2, 80, 4>::CHUNK_ROWS : 32);
+}
 
 cudaError_t launch_decode_kernel(int n_branch, const CUtensorMap& map_ckv, const CUtensorMap& map_krope,
                                  const DecodeArgs& a, int groups, cudaStream_t stream, bool pdl) {
   if (n_branch < 1 || a.d_c % n_branch != 0 || a.d_c % 128 != 0 || a.d_c > 512) return cudaErrorInvalidValue;
   switch (a.d_c / n_branch) {  // branch width
     case 128: return launch_decode_split_kernel(map_ckv, map_krope, a, groups, stream, pdl);
-    case 256: return launch_decode<2, 64, 5>(map_ckv, map_krope, a, groups, stream, pdl);
+    case 256: return launch_decode<2, 80, 4>(map_ckv, map_krope, a, groups, stream, pdl);
     case 512: return launch_decode<1, 48, 4>(map_ckv, map_krope, a, groups, stream, pdl);
     default: return cudaErrorInvalidValue;
   }
