@@ -37,6 +37,11 @@ SMALL = [
     _case("stress_mlra4", 4, (3000, 17), alpha_q=synth.A_Q_V3, alpha_kv=synth.A_KV_V3),
     _case("stress_mla", 1, (3000, 17), alpha_q=synth.A_Q_V3, alpha_kv=synth.A_KV_V3),
     _case("outlier_mlra4", 4, (5000,), outlier_frac=0.01),
+    # the tile boundaries of the 48-token MLA and 80-token MLRA-2 kernels (16-row TMA boxes)
+    _case("tails48_mla", 1, (47, 48, 49, 95, 96, 97)),
+    _case("paged32_tails48_mla", 1, (47, 49, 97, 200), page_size=32),
+    _case("tails80_mlra2", 2, (79, 80, 81, 159, 160, 161)),
+    _case("paged64_tails80_mlra2", 2, (79, 81, 161, 300), page_size=64),
 ]
 
 
