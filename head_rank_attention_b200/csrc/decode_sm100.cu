@@ -12,9 +12,10 @@
 //   blockIdx.x = slice c in 0..d_c/128-1: the CTA owns output latent columns [128c, 128c+128),
 //                which belong to branch b = c / (W/128) of width W = 512/NB;
 //   blockIdx.y = group g: a contiguous range of cache tiles (see schedule.cuh).
-// A CTA streams, for every tile of NT tokens, the branch's W latent columns plus the 64
-// RoPE columns (TMA, 64x32 boxes, 128-byte swizzle), converts them to fp16 in shared
-// memory, computes S = Q~_b [C_b | K_R]^T for all 128 head rows with tcgen05 (A = Q~
+// A CTA streams, for every tile of NT tokens (48 for MLA, 80 for 256-wide branches), the
+// branch's W latent columns plus the 64 RoPE columns (TMA, 64-column boxes of 16 rows,
+// 128-byte swizzle), converts them to fp16 in shared memory, computes
+// S = Q~_b [C_b | K_R]^T for all 128 head rows with tcgen05 (A = Q~
 // from TMEM, B = the tile, D = S in TMEM), runs the online softmax, writes P (fp16) back
 // over S in TMEM and accumulates O += P V with V = its 128 latent columns of the same
 // tile (A = P from TMEM, B = MN-major tile).  Each segment ends by writing the
