@@ -90,10 +90,16 @@ def decode_source_hash() -> str:
     return h.hexdigest()[:16]
 
 
-def ncu_traffic(workload: str):
+def traffic_key(workload: str, tp: int = 0, gla: int = 0, int8: bool = False) -> str:
+    """Key of a decode launch's recorded traffic: the workload, the shard or GLA group and the
+    cache format (each runs a different kernel or different bytes)."""
+    return workload + (f"/tp{tp}" if tp else "") + (f"/gla{gla}" if gla else "") + ("/int8" if int8 else "")
+
+
+def ncu_traffic(workload: str, path=None):
     """dram bytes per decode launch from the committed ncu summary, if it matches the
     current kernel source; else None."""
-    f = ROOT / "profiles" / "decode_dram_traffic.json"
+    f = ROOT / "profiles" / "decode_dram_traffic.json" if path is None else path
     if not f.exists():
         return None
     d = json.loads(f.read_text())
@@ -522,9 +528,7 @@ def run_native(args, wl, world, rank, local):
         achieved_gbs = kv / (decode_ms * 1e-3) / 1e9
         flops = tensor_flops_per_token(n_branch, heads, d_c) * int(lens.astype(np.int64).sum())
         achieved_tflops = flops / (decode_ms * 1e-3) / 1e12
-        # recorded per workload, shard and cache format (the int8 cache is a different kernel)
-        traffic = ncu_traffic(wl.name + (f"/tp{tpw}" if tpw else "") + (f"/gla{gla}" if gla else "")
-                              + ("/int8" if int8 else ""))
+        traffic = ncu_traffic(traffic_key(wl.name, tpw, gla, int8))
         if gla:
             parallelism = (f"gla{gla}: head-and-latent groups, outs gathered over heads" if world == gla
                            else f"gla{gla}: rank 0's group alone (no gather)")

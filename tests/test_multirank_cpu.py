@@ -158,3 +158,23 @@ def test_prefill_flop_count_matches_a_brute_count():
     L, n, h, nb = 9, 4, 3, 4
     pairs = sum(1 for j in range(n) for t in range(L) if t <= L - n + j)
     assert bench.prefill_flops(L, n, h, nb) == 4 * L * 512 * 128 * h + 2 * 320 * pairs * h * nb
+
+
+def test_recorded_traffic_is_keyed_by_shard_group_and_cache_format(tmp_path):
+    """A launch reads the traffic recorded for its own kernel and bytes: the int8 cache, a
+    branch shard or a GLA group never picks up the bf16 whole-model figure, and a record
+    taken from other kernel sources is ignored."""
+    import json
+    import bench
+    assert bench.traffic_key("paged_b64_t32k_mlra4") == "paged_b64_t32k_mlra4"
+    keys = {bench.traffic_key("w", tp=4), bench.traffic_key("w", gla=2), bench.traffic_key("w", int8=True),
+            bench.traffic_key("w", tp=4, int8=True), bench.traffic_key("w")}
+    assert len(keys) == 5
+    sha = bench.decode_source_hash()
+    rec = {"w": {"decode_source_sha": sha, "dram_bytes_per_launch": 123},
+           "w/int8": {"decode_source_sha": "0" * 16, "dram_bytes_per_launch": 45}}
+    f = tmp_path / "traffic.json"
+    f.write_text(json.dumps(rec))
+    assert bench.ncu_traffic(bench.traffic_key("w"), f) == 123
+    assert bench.ncu_traffic(bench.traffic_key("w", int8=True), f) is None   # stale source
+    assert bench.ncu_traffic(bench.traffic_key("w", tp=4), f) is None        # not recorded
