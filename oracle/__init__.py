@@ -13,7 +13,8 @@ own, so no pin compares against a number printed on the pages.
 from .reference import (rope_rotate, mlra_decode_expanded, mlra_decode_absorbed, mla_decode, gla_decode,
                         mlra_prefill_expanded,
                         mla_nope_key, mlra_nope_key_blocks, decode_batch, dequantize_int8_blocks,
-                        decode_batch_int8)
+                        decode_batch_int8, mlra_partial_state, combine_partial_states, upproject_latent)
 
 __all__ = ["rope_rotate", "mlra_decode_expanded", "mlra_decode_absorbed", "mla_decode", "gla_decode", "mlra_prefill_expanded",
-           "mla_nope_key", "mlra_nope_key_blocks", "decode_batch", "dequantize_int8_blocks", "decode_batch_int8"]
+           "mla_nope_key", "mlra_nope_key_blocks", "decode_batch", "dequantize_int8_blocks", "decode_batch_int8",
+           "mlra_partial_state", "combine_partial_states", "upproject_latent"]

@@ -347,6 +347,73 @@ def decode_batch_int8(inp, wl, q8, scale, heads=None, seqs=None) -> np.ndarray:
     return np.stack(res)
 
 
+def mlra_partial_state(q, c_kv, k_rope, w_uk, n_branch: int, pos: int, alpha_q: float = 1.0,
+                       alpha_kv: float = 1.0, softmax_scale: float | None = None,
+                       rope_theta: float = 10000.0, heads=None):
+    """The decode's state over a subset of one sequence's cached tokens, for a sequence
+    split across devices by token range.
+
+    c_kv [n, d_c] and k_rope [n, d_rope] are the subset's rows (K_R rotated at their own
+    positions); ``pos`` is the query's position, the sequence's last token, whatever the
+    subset.  For each head i and branch b, with the expanded scores of
+    ``mlra_decode_expanded`` restricted to the subset,
+      o^(b)   = sum_t softmax_t C_t^(b)        (the branch's latent columns, before W_UV)
+      lse^(b) = log2 sum_t exp(score_t)        (-inf for an empty subset, with o = 0)
+    Returns (o [len(heads), n_branch, w], lse [len(heads), n_branch]).
+    """
+    q, c_kv, k_rope, w_uk = _f64(q), _f64(c_kv), _f64(k_rope), _f64(w_uk)
+    h_all, d_qk = q.shape
+    d_c = w_uk.shape[1]
+    d_rope = k_rope.shape[1]
+    d_nope = d_qk - d_rope
+    w = d_c // n_branch
+    tau = 1.0 / math.sqrt(d_nope + d_rope) if softmax_scale is None else softmax_scale
+    heads = range(h_all) if heads is None else heads
+    o = np.zeros((len(heads), n_branch, w))
+    lse = np.full((len(heads), n_branch), -np.inf)
+    if c_kv.shape[0] == 0:
+        return o, lse
+    for row, i in enumerate(heads):
+        q_n = alpha_q * q[i, :d_nope]
+        q_r = rope_rotate(q[i, d_nope:], pos, rope_theta)
+        for b in range(n_branch):
+            cols = slice(b * w, (b + 1) * w)
+            K_nope = alpha_kv * (c_kv[:, cols] @ w_uk[i, cols, :])
+            score = tau * (np.concatenate([K_nope, k_rope], axis=1) @ np.concatenate([q_n, q_r]))
+            m = score.max()
+            e = np.exp(score - m)
+            o[row, b] = e @ c_kv[:, cols] / e.sum()
+            lse[row, b] = (m + math.log(e.sum())) / math.log(2.0)
+    return o, lse
+
+
+def combine_partial_states(states):
+    """Merge partial states of disjoint token subsets of one sequence: with
+    m = max_r lse_r, weight_r = 2^(lse_r - m) (each subset's share of the softmax
+    denominator), o = sum_r weight_r o_r / sum_r weight_r and lse = m + log2 sum_r weight_r.
+    ``states`` is a list of (o, lse) from ``mlra_partial_state``."""
+    o = np.stack([s[0] for s in states])        # [R, h, nb, w]
+    lse = np.stack([s[1] for s in states])      # [R, h, nb]
+    m = lse.max(axis=0)
+    wts = np.where(np.isfinite(lse), 2.0 ** (lse - m), 0.0)
+    den = wts.sum(axis=0)
+    return (wts[..., None] * o).sum(axis=0) / den[..., None], m + np.log2(den)
+
+
+def upproject_latent(o, w_uv, alpha_kv: float = 1.0, branch_scale: float | None = None, heads=None):
+    """Step 3 of the decode (方法步骤详情) on latent outputs o [len(heads), n_branch, w]:
+    out^(i) = sigma_o alpha_kv sum_b o^(b),(i) W_UV^(b),(i)."""
+    w_uv = _f64(w_uv)
+    n_branch, w = o.shape[1], o.shape[2]
+    sigma = 1.0 / math.sqrt(n_branch) if branch_scale is None else branch_scale
+    heads = range(w_uv.shape[0]) if heads is None else heads
+    out = np.zeros((len(heads), w_uv.shape[2]))
+    for row, i in enumerate(heads):
+        for b in range(n_branch):
+            out[row] += o[row, b] @ w_uv[i, b * w:(b + 1) * w, :]
+    return sigma * alpha_kv * out
+
+
 def decode_batch(inp, wl, heads=None, seqs=None, form: str = "absorbed") -> np.ndarray:
     """Run the oracle over sequences of a synth.Inputs; returns [len(seqs), len(heads), d_v]."""
     from synth import logical_rows, D_C

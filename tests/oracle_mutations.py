@@ -34,6 +34,13 @@ MUTATIONS = [
     ("decode_batch_int8", "astype(np.int64) * P + t % P", "astype(np.int64) * P", "int8 cache page offset dropped"),
     ("mlra_prefill_expanded", "rope_rotate(q[j, i, d_nope:], int(pos[j]), rope_theta)",
      "rope_rotate(q[j, i, d_nope:], L - 1, rope_theta)", "every query rotated to the last position"),
+    ("mlra_partial_state", "rope_rotate(q[i, d_nope:], pos, rope_theta)",
+     "rope_rotate(q[i, d_nope:], c_kv.shape[0] - 1, rope_theta)", "a range's query rotated at the range's end"),
+    ("mlra_partial_state", "(m + math.log(e.sum())) / math.log(2.0)", "m + math.log(e.sum())",
+     "partial log-sum-exp in natural-log units"),
+    ("combine_partial_states", "2.0 ** (lse - m)", "np.exp(lse - m)", "partial weights taken with exp, not 2^"),
+    ("combine_partial_states", "(wts[..., None] * o).sum(axis=0) / den[..., None]", "o.mean(axis=0)",
+     "partial states averaged, not weighted"),
 ]
 
 

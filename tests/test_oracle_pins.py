@@ -405,3 +405,58 @@ def test_int8_decode_on_integer_cache_equals_bf16_decode(page_size):
     got = oracle.decode_batch_int8(inp, wl, q8.numpy(), s.numpy())
     ref = oracle.decode_batch(inp, wl)
     assert _rel(got, ref) < 1e-12
+
+
+# ---- a sequence split by token range (partial states and their combination) ---------------
+
+def _cp_case(seed=5, h=3, L=61):
+    rng = np.random.default_rng(seed)
+    q = rng.standard_normal((h, 192))
+    C = rng.standard_normal((L, 512))
+    KR = rng.standard_normal((L, 64))
+    wk = rng.standard_normal((h, 512, 128)) / 16
+    wv = rng.standard_normal((h, 512, 128)) / 16
+    return q, C, KR, wk, wv
+
+
+@pytest.mark.parametrize("n_branch", [1, 2, 4])
+@pytest.mark.parametrize("cuts", [(0, 61), (0, 20, 61), (0, 1, 30, 30, 60, 61), (0, 15, 31, 46, 61)])
+def test_partial_states_combine_to_the_whole_sequence_decode(n_branch, cuts):
+    """Decoding disjoint token ranges against the query at the sequence's last position and
+    merging the states by their log-sum-exp gives the decode of the whole sequence (the
+    softmax denominator is the sum of the ranges' denominators); empty ranges included."""
+    q, C, KR, wk, wv = _cp_case()
+    L = C.shape[0]
+    full = oracle.mlra_decode_expanded(q, C, KR, wk, wv, n_branch, alpha_q=1.2, alpha_kv=0.8)
+    parts = [oracle.mlra_partial_state(q, C[a:b], KR[a:b], wk, n_branch, L - 1, alpha_q=1.2, alpha_kv=0.8)
+             for a, b in zip(cuts[:-1], cuts[1:])]
+    o, lse = oracle.combine_partial_states(parts)
+    np.testing.assert_allclose(oracle.upproject_latent(o, wv, alpha_kv=0.8), full, rtol=0, atol=1e-12)
+    whole = oracle.mlra_partial_state(q, C, KR, wk, n_branch, L - 1, alpha_q=1.2, alpha_kv=0.8)
+    np.testing.assert_allclose(lse, whole[1], rtol=0, atol=1e-12)
+
+
+def test_partial_state_of_one_token_closed_form():
+    """Over a single token t the softmax is 1: o^(b) = C_t^(b), and lse^(b) is the token's
+    score in log2 units, tau (q~ . k_t) / ln 2, computed here from the expanded key."""
+    q, C, KR, wk, _ = _cp_case(h=2)
+    L, t, tau = C.shape[0], 17, 1.0 / math.sqrt(192)
+    o, lse = oracle.mlra_partial_state(q, C[t:t + 1], KR[t:t + 1], wk, 4, L - 1)
+    for i in range(2):
+        q_r = oracle.rope_rotate(q[i, 128:], L - 1)
+        for b in range(4):
+            cols = slice(128 * b, 128 * b + 128)
+            np.testing.assert_array_equal(o[i, b], C[t, cols])
+            k = np.concatenate([C[t, cols] @ wk[i, cols, :], KR[t]])
+            assert abs(lse[i, b] - tau * (k @ np.concatenate([q[i, :128], q_r])) / math.log(2.0)) < 1e-12
+
+
+def test_empty_partial_state_carries_no_weight():
+    q, C, KR, wk, wv = _cp_case()
+    L = C.shape[0]
+    empty = oracle.mlra_partial_state(q, C[:0], KR[:0], wk, 4, L - 1)
+    assert np.all(empty[1] == -np.inf) and np.all(empty[0] == 0)
+    whole = oracle.mlra_partial_state(q, C, KR, wk, 4, L - 1)
+    o, lse = oracle.combine_partial_states([empty, whole, empty])
+    np.testing.assert_allclose(o, whole[0], rtol=0, atol=1e-15)
+    np.testing.assert_allclose(lse, whole[1], rtol=0, atol=1e-15)
