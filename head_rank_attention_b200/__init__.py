@@ -9,13 +9,15 @@ device memory, streams and the process group.  Build the library with
 """
 from ._binding import (EXPORTS, HRA_BF16, HRA_F32, HRA_INT8, HraDecodeParams, HraError, HraPrefillParams, LIB_PATH,
                        alloc_prefill_workspace, alloc_workspace, check_device_status, check_prefill_status,
+                       combine_partials,
                        last_error, load_library, make_params, make_prefill_params, mla_decode, mlra_decode,
                        mlra_decode_static, mlra_prefill, prefill_workspace_size,
                        selftest_wait_timeout, version, workspace_size)
-from . import tp
+from . import cp, tp
 
 __all__ = ["EXPORTS", "HRA_BF16", "HRA_F32", "HRA_INT8", "HraDecodeParams", "HraError", "HraPrefillParams",
            "LIB_PATH", "alloc_prefill_workspace", "alloc_workspace", "check_device_status", "check_prefill_status",
+           "combine_partials", "cp",
            "last_error", "load_library", "make_params", "make_prefill_params", "mla_decode", "mlra_decode",
            "mlra_decode_static", "mlra_prefill", "prefill_workspace_size",
            "selftest_wait_timeout", "tp", "version", "workspace_size"]

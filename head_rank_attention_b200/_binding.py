@@ -27,7 +27,7 @@ STATUS_NAMES = {0: "HRA_OK", -1: "HRA_ERR_INVALID_ARG", -2: "HRA_ERR_UNSUPPORTED
 # Symbols declared in include/hra.h.
 EXPORTS = ("hra_workspace_size", "mlra_decode", "mla_decode", "mlra_decode_static", "hra_check_device_status",
            "hra_selftest_wait_timeout", "hra_last_error", "hra_version", "hra_prefill_workspace_size", "mlra_prefill",
-           "hra_check_prefill_status")
+           "hra_check_prefill_status", "hra_combine_partials")
 
 
 class HraError(RuntimeError):
@@ -54,6 +54,7 @@ class HraDecodeParams(ctypes.Structure):
         ("stage_events", ctypes.c_void_p),
         ("out_accumulate", ctypes.c_int), ("n_out_peers", ctypes.c_int), ("out_peers", ctypes.c_void_p),
         ("cache_dtype", ctypes.c_int), ("ckv_scale", ctypes.c_void_p), ("ckv_scale_stride", ctypes.c_int64),
+        ("q_positions", ctypes.c_void_p), ("part_o", ctypes.c_void_p), ("part_lse", ctypes.c_void_p),
     ]
 
 
@@ -97,6 +98,8 @@ def load_library() -> ctypes.CDLL:
     for name in ("mlra_prefill", "hra_check_prefill_status"):
         getattr(lib, name).argtypes = [PP, ctypes.c_void_p]
         getattr(lib, name).restype = ctypes.c_int
+    lib.hra_combine_partials.argtypes = [P, ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p]
+    lib.hra_combine_partials.restype = ctypes.c_int
     lib.hra_selftest_wait_timeout.argtypes = [ctypes.c_void_p, ctypes.c_int, ctypes.c_void_p]
     lib.hra_selftest_wait_timeout.restype = ctypes.c_int
     lib.hra_last_error.argtypes = []
@@ -136,14 +139,17 @@ def make_params(q, ckv, krope, seq_lens, w_uk, w_uv, out, workspace=None, *, n_b
                 softmax_scale: float = 0.0, rope_theta: float = 10000.0, block_table=None,
                 page_size: int = 0, seq_stride: int = 0, cache_rows: Optional[int] = None,
                 num_splits: int = 0, wait_limit: int = 0, out_accumulate: bool = False,
-                out_peers=None, ckv_scale=None) -> HraDecodeParams:
+                out_peers=None, ckv_scale=None, q_positions=None, part_o=None,
+                part_lse=None) -> HraDecodeParams:
     """Fill hra_decode_params from torch tensors (shapes/dtypes as documented in hra.h).
 
     ckv / krope are 2-D row views of the cache (e.g. cache[:, :512], cache[:, 512:]);
     their row strides become ckv_stride / krope_stride.  An int8 ckv selects the quantised
     cache: ckv_scale is then the fp32 [rows, d_c / 128] view of its block scales.  out_peers: device addresses (ints)
     or tensors of other ranks' out buffers for out_accumulate (the array is kept alive on
-    the returned object).
+    the returned object).  q_positions (int32 [B]), part_o (fp32 [B, h, d_c]) and part_lse
+    (fp32 [B, h, d_c / 128]) make the call the decode of one token range of longer
+    sequences (see hra.h); out may then be None.
     """
     import torch
     p = HraDecodeParams()
@@ -177,6 +183,7 @@ def make_params(q, ckv, krope, seq_lens, w_uk, w_uv, out, workspace=None, *, n_b
     p._out_peers = (ctypes.c_void_p * max(1, len(peers)))(*peers)
     p.out_peers = ctypes.cast(p._out_peers, ctypes.c_void_p).value if peers else None
     p.n_out_peers = len(peers)
+    p.q_positions, p.part_o, p.part_lse = _ptr(q_positions), _ptr(part_o), _ptr(part_lse)
     return p
 
 
@@ -199,6 +206,14 @@ def mlra_decode_static(p: HraDecodeParams, stream=None) -> None:
     """Decode without a workspace (scratch from the library's 32 MiB static device array):
     for callers that cannot allocate device memory.  p.workspace is ignored."""
     _check(load_library().mlra_decode_static(ctypes.byref(p), ctypes.c_void_p(_stream_handle(stream))))
+
+
+def combine_partials(p: HraDecodeParams, parts_o, parts_lse, stream=None) -> None:
+    """Merge the gathered token-range states parts_o (fp32 [n, B, h, d_c]) and parts_lse
+    (fp32 [n, B, h, d_c / 128]) and finish the decode into p.out (hra_combine_partials)."""
+    _check(load_library().hra_combine_partials(ctypes.byref(p), int(parts_o.shape[0]), ctypes.c_void_p(_ptr(parts_o)),
+                                               ctypes.c_void_p(_ptr(parts_lse)),
+                                               ctypes.c_void_p(_stream_handle(stream))))
 
 
 def check_device_status(p: HraDecodeParams, stream=None) -> None:

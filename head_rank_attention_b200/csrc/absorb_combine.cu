@@ -136,12 +136,12 @@ absorb_tc_kernel(const __grid_constant__ CUtensorMap map_wuk, const __grid_const
   const int part = warp >> 2;            // columns [256 nh + 128 part, +128); rope pairs [16 part, +16)
   const long long row = (static_cast<long long>(s) * a.heads + i) * (dc + 64);
   if (s < a.batch && nh == 0) {
-    // RoPE of the query's rope part at position L-1, while the loads and MMAs run: pair
-    // (j, j + 32) turns by pos * theta^(-2j/64) radians.  The angle is carried in turns
-    // (fp64: pos reaches 2^21); its fractional part is exact and is then evaluated in
-    // fp32 by sincospif.
+    // RoPE of the query's rope part at position L-1 (or the caller's q_positions[s], for a
+    // token range of a longer sequence), while the loads and MMAs run: pair (j, j + 32)
+    // turns by pos * theta^(-2j/64) radians.  The angle is carried in turns (fp64: pos
+    // reaches 2^21); its fractional part is exact and is then evaluated in fp32 by sincospif.
     const int L = a.seq_lens[s];
-    const double pos = static_cast<double>(L > 0 ? L - 1 : 0);
+    const double pos = static_cast<double>(a.q_positions != nullptr ? max(a.q_positions[s], 0) : (L > 0 ? L - 1 : 0));
     const uint4* qr = reinterpret_cast<const uint4*>(a.q + (static_cast<long long>(s) * a.heads + i) * 192 + 128);
     __align__(16) __nv_bfloat16 x1[16], x2[16];
     *reinterpret_cast<uint4*>(x1) = qr[2 * part];
@@ -218,7 +218,7 @@ __device__ __forceinline__ bool group_live(int g, int G, int T) {
 // consecutive latent columns of the slice); the Z thread sets take alternate runs of GU
 // groups and are merged through shared memory at the end.  Every load of a run of GU
 // groups is issued before any of them is used.
-template <int CPT, int Z, int GU>
+template <int CPT, int Z, int GU, bool PARTIAL = false>
 __global__ void __launch_bounds__(256 * Z) merge_kernel(const CombineArgs a) {
   constexpr int TPH = 128 / CPT;    // threads per head
   constexpr int HPB = 256 / TPH;    // heads per block
@@ -294,9 +294,21 @@ __global__ void __launch_bounds__(256 * Z) merge_kernel(const CombineArgs a) {
 #pragma unroll
       for (int u = 0; u < CPT; ++u) acc[u] = acc[u] * r0 + xchg[t][2 + u] * r1;
     }
+    M = mx;  // den and acc are now relative to the larger maximum
   }
   if (head >= a.heads) return;
   const float inv = den > 0.f ? 1.f / den : 0.f;  // an empty sequence gives zeros
+  if constexpr (PARTIAL) {
+    // the state of this token range: the normalised latent row and log2 of its softmax
+    // denominator (sum_t 2^(score_t log2 e) = 2^M * den)
+    const long long hs = static_cast<long long>(seq) * a.heads + head;
+    float4* dst = reinterpret_cast<float4*>(a.part_o + hs * a.d_c + 128 * slice + col);
+#pragma unroll
+    for (int v = 0; v < CPT / 4; ++v)
+      dst[v] = make_float4(acc[4 * v] * inv, acc[4 * v + 1] * inv, acc[4 * v + 2] * inv, acc[4 * v + 3] * inv);
+    if (col == 0) a.part_lse[hs * gridDim.y + slice] = den > 0.f ? M + log2f(den) : -INFINITY;
+    return;
+  }
   // o_lat as hi / lo bf16 terms, [h][B][d_c] each
   const long long base = (static_cast<long long>(head) * a.batch + seq) * a.d_c + 128 * slice + col;
   __align__(16) __nv_bfloat16 hi[CPT], lo[CPT];
@@ -681,6 +693,62 @@ __global__ void __launch_bounds__(kSmallThreads, 2) combine_small_kernel(const C
   cluster.sync();  // the other slices keep their shared memory until rank 0 has read it
 }
 
+// ---------------------------------------------------------------------------- partial states
+// hra_combine_partials: grid (ceil(h / 32), d_c / 128 slices, B), 256 threads; thread =
+// (head, 16 consecutive latent columns of the slice).  Merges the a.n_parts states of its
+// (sequence, head, slice) by their log2 softmax denominators and writes the merged row as
+// o_lat's hi / lo bf16 terms, which the up-projection then reads.
+__global__ void __launch_bounds__(256) partial_combine_kernel(const CombineArgs a) {
+  constexpr int CPT = 16;
+  if (threadIdx.x == 0) grid_dep_launch();
+  grid_dep_wait();  // o_lat is read by the previous call's up-projection
+  const int head = blockIdx.x * 32 + threadIdx.x / 8;
+  const int col = (threadIdx.x % 8) * CPT;
+  const int slice = blockIdx.y, seq = blockIdx.z, slices = gridDim.y;
+  if (head >= a.heads) return;
+  const long long hs = static_cast<long long>(seq) * a.heads + head;
+  const long long part_o = static_cast<long long>(a.batch) * a.heads * a.d_c;     // elements per part
+  const long long part_l = static_cast<long long>(a.batch) * a.heads * slices;
+  float m = -INFINITY;
+  for (int r = 0; r < a.n_parts; ++r) m = fmaxf(m, a.parts_lse[r * part_l + hs * slices + slice]);
+  float acc[CPT];
+#pragma unroll
+  for (int u = 0; u < CPT; ++u) acc[u] = 0.f;
+  float wsum = 0.f;
+  if (m != -INFINITY) {
+    for (int r = 0; r < a.n_parts; ++r) {
+      const float lse = a.parts_lse[r * part_l + hs * slices + slice];
+      if (lse == -INFINITY) continue;
+      const float wt = exp2f(lse - m);
+      wsum += wt;
+      const float4* src = reinterpret_cast<const float4*>(a.parts_o + r * part_o + hs * a.d_c + 128 * slice + col);
+#pragma unroll
+      for (int v = 0; v < CPT / 4; ++v) {
+        const float4 x = src[v];
+        acc[4 * v + 0] = fmaf(wt, x.x, acc[4 * v + 0]);
+        acc[4 * v + 1] = fmaf(wt, x.y, acc[4 * v + 1]);
+        acc[4 * v + 2] = fmaf(wt, x.z, acc[4 * v + 2]);
+        acc[4 * v + 3] = fmaf(wt, x.w, acc[4 * v + 3]);
+      }
+    }
+  }
+  const float inv = wsum > 0.f ? 1.f / wsum : 0.f;  // every range empty: zeros
+  const long long base = (static_cast<long long>(head) * a.batch + seq) * a.d_c + 128 * slice + col;
+  __align__(16) __nv_bfloat16 hi[CPT], lo[CPT];
+#pragma unroll
+  for (int u = 0; u < CPT; ++u) {
+    const float x = acc[u] * inv;
+    hi[u] = __float2bfloat16_rn(x);
+    lo[u] = __float2bfloat16_rn(x - __bfloat162float(hi[u]));
+  }
+  __nv_bfloat16* lo_base = a.o_lat + static_cast<long long>(a.heads) * a.batch * a.d_c;
+#pragma unroll
+  for (int v = 0; v < CPT / 8; ++v) {
+    *reinterpret_cast<uint4*>(a.o_lat + base + 8 * v) = reinterpret_cast<const uint4*>(hi)[v];
+    *reinterpret_cast<uint4*>(lo_base + base + 8 * v) = reinterpret_cast<const uint4*>(lo)[v];
+  }
+}
+
 template <class K>
 cudaError_t set_smem(K kern, int bytes) {
   return cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
@@ -706,6 +774,13 @@ cudaError_t launch_combine_upproj(const CUtensorMap& map_wuv, const CUtensorMap&
   // set for up to 64 groups: used where that grid fits on the SMs at once.  With more heads
   // or groups the merge kernel and the tensor-core up-projection are faster (measured at
   // h = 128 with 37 and 148 groups).
+  if (a.part_o != nullptr) {  // partial mode: the merged states are the call's output
+    if (a.batch >= 16)
+      return launch_kernel(merge_kernel<16, 1, 2, true>, dim3((a.heads + 31) / 32, a.d_c / 128, a.batch), dim3(256),
+                           0, stream, pdl, a);
+    return launch_kernel(merge_kernel<4, 2, 4, true>, dim3((a.heads + 7) / 8, a.d_c / 128, a.batch), dim3(512), 0,
+                         stream, pdl, a);
+  }
   if (a.batch <= kSmallBatch && (a.d_c / 128) * a.heads <= a.sms && a.groups <= 64)
     return launch_kernel_cluster(combine_small_kernel, dim3(a.d_c / 128, a.heads), dim3(kSmallThreads), 0, stream, pdl,
                                  a.d_c / 128, a);
@@ -718,6 +793,16 @@ cudaError_t launch_combine_upproj(const CUtensorMap& map_wuv, const CUtensorMap&
   else
     e = launch_kernel(merge_kernel<4, 2, 4>, dim3((a.heads + 7) / 8, a.d_c / 128, a.batch), dim3(512), 0, stream,
                       pdl, a);
+  if (e != cudaSuccess) return e;
+  if ((e = set_smem(upproj_tc_kernel, UpprojCfg::SMEM)) != cudaSuccess) return e;
+  return launch_kernel(upproj_tc_kernel, dim3(a.heads, (a.batch + 127) / 128), dim3(UpprojCfg::THREADS),
+                       UpprojCfg::SMEM, stream, pdl, map_wuv, map_olat, a);
+}
+
+cudaError_t launch_combine_partials(const CUtensorMap& map_wuv, const CUtensorMap& map_olat, const CombineArgs& a,
+                                    cudaStream_t stream, bool pdl) {
+  cudaError_t e = launch_kernel(partial_combine_kernel, dim3((a.heads + 31) / 32, a.d_c / 128, a.batch), dim3(256),
+                                0, stream, pdl, a);
   if (e != cudaSuccess) return e;
   if ((e = set_smem(upproj_tc_kernel, UpprojCfg::SMEM)) != cudaSuccess) return e;
   return launch_kernel(upproj_tc_kernel, dim3(a.heads, (a.batch + 127) / 128), dim3(UpprojCfg::THREADS),

@@ -19,6 +19,7 @@ struct AbsorbArgs {
   int batch, heads;
   int d_c;                    // latent width: 512, or 256 / 128 (a shard of 128-wide branches)
   float alpha_q, alpha_kv, rope_theta;
+  const int32_t* q_positions; // [B] query position per sequence, or nullptr: seq_lens[s] - 1
 };
 
 constexpr int kMaxOutPeers = 7;  // other ranks' out buffers the up-projection can add into
@@ -39,6 +40,14 @@ struct CombineArgs {
   int d_c;                    // latent width (as in AbsorbArgs)
   int sms;                    // streaming multiprocessors of the device
   float alpha_kv, branch_scale;
+  // partial mode: the merge writes fp32 [B, h, d_c] normalised latent rows and fp32
+  // [B, h, d_c / 128] log2 softmax denominators here, and nothing runs after it
+  float* part_o;
+  float* part_lse;
+  // hra_combine_partials: n_parts gathered states [n_parts, B, h, d_c] / [n_parts, B, h, d_c / 128]
+  const float* parts_o;
+  const float* parts_lse;
+  int n_parts;
 };
 
 // Sequences per absorb CTA (the MMA's M); the q tensor map's box is {64, this} rows.
@@ -58,5 +67,9 @@ constexpr int kSmallBatch = 4;
 // map_olat: a.o_lat viewed as [2*h*B rows, d_c] bf16, box {64, upproj_seq_chunk()}, SWIZZLE_128B.
 cudaError_t launch_combine_upproj(const CUtensorMap& map_wuv, const CUtensorMap& map_olat, const CombineArgs& a,
                                   cudaStream_t stream, bool pdl);
+// Merge a.n_parts gathered partial states (a.parts_o / a.parts_lse) into o_lat and run the
+// up-projection (hra_combine_partials).
+cudaError_t launch_combine_partials(const CUtensorMap& map_wuv, const CUtensorMap& map_olat, const CombineArgs& a,
+                                    cudaStream_t stream, bool pdl);
 
 }  // namespace hra

@@ -80,13 +80,21 @@ hra_status validate(const hra_decode_params* p) {
     return fail(HRA_ERR_UNSUPPORTED, "batch=%d (supported: 1..%d)", p->batch, hra::kMaxBatch);
   if (p->num_heads < 1 || p->num_heads > 128)
     return fail(HRA_ERR_UNSUPPORTED, "num_heads=%d (supported: 1..128)", p->num_heads);
+  // partial mode (a token range of a split sequence): the merged states go to part_o /
+  // part_lse and out is not used
+  const bool partial = p->part_o != nullptr || p->part_lse != nullptr;
+  if (partial && (p->part_o == nullptr || p->part_lse == nullptr))
+    return fail(HRA_ERR_INVALID_ARG, "part_o and part_lse must both be set (or both NULL)");
   const struct { const void* ptr; const char* name; } ptrs[] = {
       {p->q, "q"}, {p->ckv, "ckv"}, {p->krope, "krope"}, {p->seq_lens, "seq_lens"},
-      {p->w_uk, "w_uk"}, {p->w_uv, "w_uv"}, {p->out, "out"}};
+      {p->w_uk, "w_uk"}, {p->w_uv, "w_uv"}, {partial ? p->part_o : p->out, partial ? "part_o" : "out"},
+      {partial ? p->part_lse : p->w_uv, "part_lse"}};
   for (const auto& x : ptrs) {
     if (x.ptr == nullptr) return fail(HRA_ERR_INVALID_ARG, "%s is NULL", x.name);
     if (!aligned16(x.ptr)) return fail(HRA_ERR_INVALID_ARG, "%s is not 16-byte aligned", x.name);
   }
+  if (p->q_positions != nullptr && (reinterpret_cast<uintptr_t>(p->q_positions) & 3u) != 0)
+    return fail(HRA_ERR_INVALID_ARG, "q_positions is not 4-byte aligned");
   if (p->ckv_stride < p->d_c || p->ckv_stride % 8 != 0)
     return fail(HRA_ERR_INVALID_ARG, "ckv_stride=%lld must be >= d_c=%d and a multiple of 8",
                 (long long)p->ckv_stride, p->d_c);
@@ -258,6 +266,7 @@ hra_status run_decode(const hra_decode_params* p, cudaStream_t stream) {
   ab.d_c = dc;
   ab.tile_prefix = tile_prefix;
   ab.tile_tokens = hra::decode_tile_tokens(dc / p->n_branch);
+  ab.q_positions = p->q_positions;
   // Programmatic dependent launch lets each kernel start while the previous one drains;
   // the stage-timing mode launches plainly so that its events bracket whole kernels.
   const bool pdl = p->stage_events == nullptr;
@@ -307,11 +316,71 @@ hra_status run_decode(const hra_decode_params* p, cudaStream_t stream) {
   cb.groups = plan.groups;
   cb.d_c = dc;
   if ((st = sm_count(&cb.sms)) != HRA_OK) return st;
+  cb.part_o = p->part_o;
+  cb.part_lse = p->part_lse;
   cb.alpha_kv = p->alpha_kv;
   cb.branch_scale = p->branch_scale;
   e = hra::launch_combine_upproj(map_wuv, map_olat, cb, stream, pdl);
   if (e != cudaSuccess) return cuda_fail(e, "combine_upproj launch");
   if ((e = mark(3)) != cudaSuccess) return cuda_fail(e, "stage event");
+  g_last_error.clear();
+  return HRA_OK;
+}
+
+// Merge the gathered states of a sequence split by token range, then the up-projection
+// (hra_combine_partials).
+constexpr int kMaxParts = 64;
+
+hra_status run_combine_partials(const hra_decode_params* p, int n_parts, const float* parts_o, const float* parts_lse,
+                                cudaStream_t stream) {
+  if (p == nullptr) return fail(HRA_ERR_INVALID_ARG, "params is NULL");
+  hra_decode_params q = *p;  // the decode's parameters, finishing into out
+  q.part_o = nullptr;
+  q.part_lse = nullptr;
+  hra_status st = validate(&q);
+  if (st != HRA_OK) return st;
+  if (n_parts < 1 || n_parts > kMaxParts)
+    return fail(HRA_ERR_INVALID_ARG, "n_parts=%d (supported: 1..%d)", n_parts, kMaxParts);
+  if (parts_o == nullptr || parts_lse == nullptr || !aligned16(parts_o) || !aligned16(parts_lse))
+    return fail(HRA_ERR_INVALID_ARG, "parts_o / parts_lse NULL or not 16-byte aligned");
+  Plan plan;
+  if ((st = make_plan(&q, &plan)) != HRA_OK) return st;
+  if (q.workspace == nullptr) return fail(HRA_ERR_WORKSPACE, "workspace is NULL");
+  if ((reinterpret_cast<uintptr_t>(q.workspace) & 255u) != 0)
+    return fail(HRA_ERR_WORKSPACE, "workspace is not 256-byte aligned");
+  if (q.workspace_bytes < plan.total)
+    return fail(HRA_ERR_WORKSPACE, "workspace_bytes=%zu < required %zu", q.workspace_bytes, plan.total);
+  uint8_t* ws = static_cast<uint8_t*>(q.workspace);
+  int* status = reinterpret_cast<int*>(ws);
+  __nv_bfloat16* o_lat = reinterpret_cast<__nv_bfloat16*>(ws + plan.o_lat);
+  const int h = q.num_heads, B = q.batch, dc = q.d_c;
+  CUtensorMap map_wuv, map_olat;
+  if ((st = encode_map(&map_wuv, q.w_uv, 128, static_cast<int64_t>(h) * dc, 128, 128)) != HRA_OK) return st;
+  if ((st = encode_map(&map_olat, o_lat, dc, 2 * static_cast<int64_t>(h) * B, dc, hra::upproj_seq_chunk())) !=
+      HRA_OK)
+    return st;
+  cudaError_t e = cudaMemsetAsync(status, 0, 4 * sizeof(int), stream);
+  if (e != cudaSuccess) return cuda_fail(e, "status clear");
+  hra::CombineArgs cb{};
+  cb.o_lat = o_lat;
+  cb.w_uv = static_cast<const __nv_bfloat16*>(q.w_uv);
+  cb.status = status;
+  cb.out_f32 = q.out_dtype == HRA_F32 ? static_cast<float*>(q.out) : nullptr;
+  cb.out_bf16 = q.out_dtype == HRA_BF16 ? static_cast<__nv_bfloat16*>(q.out) : nullptr;
+  cb.accumulate = q.out_accumulate;
+  cb.n_peers = q.n_out_peers;
+  for (int k = 0; k < q.n_out_peers; ++k) cb.peers[k] = static_cast<float*>(q.out_peers[k]);
+  cb.batch = B;
+  cb.heads = h;
+  cb.groups = plan.groups;
+  cb.d_c = dc;
+  cb.alpha_kv = q.alpha_kv;
+  cb.branch_scale = q.branch_scale;
+  cb.parts_o = parts_o;
+  cb.parts_lse = parts_lse;
+  cb.n_parts = n_parts;
+  e = hra::launch_combine_partials(map_wuv, map_olat, cb, stream, true);
+  if (e != cudaSuccess) return cuda_fail(e, "combine_partials launch");
   g_last_error.clear();
   return HRA_OK;
 }
@@ -494,6 +563,11 @@ hra_status mla_decode(const hra_decode_params* p, void* stream) {
   if (p != nullptr && p->n_branch != 1)
     return fail(HRA_ERR_INVALID_ARG, "mla_decode requires n_branch == 1 (got %d)", p->n_branch);
   return run_decode(p, static_cast<cudaStream_t>(stream));
+}
+
+hra_status hra_combine_partials(const hra_decode_params* p, int n_parts, const float* parts_o, const float* parts_lse,
+                                void* stream) {
+  return run_combine_partials(p, n_parts, parts_o, parts_lse, static_cast<cudaStream_t>(stream));
 }
 
 hra_status hra_check_device_status(const hra_decode_params* p, void* stream) {

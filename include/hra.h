@@ -148,6 +148,19 @@ typedef struct {
   hra_dtype cache_dtype;        /* HRA_BF16 (default) or HRA_INT8                          */
   const float* ckv_scale;       /* fp32 scales, row r's at ckv_scale + r * ckv_scale_stride */
   int64_t ckv_scale_stride;     /* floats between consecutive rows' scales, >= d_c / 128   */
+
+  /* One sequence split across devices by token range (optional; NULL = off).  A device
+     holding tokens [a, b) of a sequence of L tokens passes its rows as the sequence
+     (seq_lens[s] = b - a) and q_positions[s] = L - 1, the query's position; with part_o
+     and part_lse set the call stops after the split-KV merge and writes, for every
+     (sequence, head, 128-column slice of the latent), the slice's softmax-weighted latent
+     row over its tokens (normalised) and the log2 of the slice's softmax denominator
+     (log2 sum_t exp(score_t); -inf for an empty range, with a zero row).  out is then
+     neither read nor written (it may be NULL).  The devices gather these states and one
+     hra_combine_partials call merges them and finishes the decode.                      */
+  const int32_t* q_positions;   /* [B] position of each sequence's query, or NULL: L - 1   */
+  float* part_o;                /* fp32 [B, h, d_c], 16-B aligned, or NULL                 */
+  float* part_lse;              /* fp32 [B, h, d_c / 128], 16-B aligned, or NULL           */
 } hra_decode_params;
 
 /* Bytes of workspace one call with these parameters needs (0 on invalid parameters).
@@ -177,6 +190,19 @@ HRA_API hra_status mla_decode(const hra_decode_params* p, void* stream /* cudaSt
  * race; the status word is cleared by every call, and expired device waits recorded there
  * are not reachable through hra_check_device_status.  Allocates nothing. */
 HRA_API hra_status mlra_decode_static(const hra_decode_params* p, void* stream /* cudaStream_t */);
+
+/* Finish a decode whose tokens were split into n_parts ranges (across devices, see
+ * q_positions / part_o / part_lse above): parts_o fp32 [n_parts, B, h, d_c] and parts_lse
+ * fp32 [n_parts, B, h, d_c / 128] hold the ranges' states in any order (device memory,
+ * 16-B aligned; an all-gather of every device's part_o / part_lse produces them).  Per
+ * (sequence, head, slice) the states are merged by their log-sum-exp (with m the largest
+ * lse, each range's row is weighted by 2^(lse - m) and the weights' sum normalises), and
+ * the merged latent rows go through the up-projection and branch sum of mlra_decode into
+ * p->out (out_dtype, out_accumulate and out_peers as there).  p is the decode's parameter
+ * block: shapes, w_uv, alpha_kv, branch_scale, out and a workspace of
+ * hra_workspace_size(p) bytes; its part_o and part_lse are ignored.  1 <= n_parts <= 64. */
+HRA_API hra_status hra_combine_partials(const hra_decode_params* p, int n_parts, const float* parts_o,
+                                        const float* parts_lse, void* stream /* cudaStream_t */);
 
 /*
  * Prefill: causal multi-token MLRA for one sequence, in the expanded form ("vllbc02MLA":

@@ -249,3 +249,49 @@ def test_prefill_workspace_size_formula():
     expect = r(expect + 4 * 16 * l_pad * 128 * 2)
     assert hra.prefill_workspace_size(p) == expect
     assert hra.load_library().hra_prefill_workspace_size(ctypes.byref(_fake_prefill(n_branch=5))) == 0
+
+
+@pytest.mark.parametrize("over,status", [
+    (dict(part_o=0xB0000), B.HRA_ERR_INVALID_ARG),                        # part_lse missing
+    (dict(part_lse=0xC0000), B.HRA_ERR_INVALID_ARG),                      # part_o missing
+    (dict(part_o=0xB0008, part_lse=0xC0000), B.HRA_ERR_INVALID_ARG),      # misaligned
+    (dict(q_positions=0xD0002), B.HRA_ERR_INVALID_ARG),                   # misaligned
+    (dict(part_o=0xB0000, part_lse=0xC0000, out=None), B.HRA_ERR_WORKSPACE),  # well formed: out unused
+    (dict(q_positions=0xD0000), B.HRA_ERR_WORKSPACE),
+])
+def test_token_range_fields_are_validated(over, status):
+    """The token-range mode of a split sequence (q_positions, part_o, part_lse) is checked
+    before any launch; in it out may be NULL."""
+    p = _fake_params(**over)
+    rc = hra.load_library().mlra_decode(ctypes.byref(p), None)
+    assert rc == status, hra.last_error()
+
+
+@pytest.mark.parametrize("n_parts,parts_o,parts_lse,over,status", [
+    (0, 0xB0000, 0xC0000, {}, B.HRA_ERR_INVALID_ARG),
+    (65, 0xB0000, 0xC0000, {}, B.HRA_ERR_INVALID_ARG),
+    (2, None, 0xC0000, {}, B.HRA_ERR_INVALID_ARG),
+    (2, 0xB0004, 0xC0000, {}, B.HRA_ERR_INVALID_ARG),
+    (2, 0xB0000, 0xC0000, dict(out=None), B.HRA_ERR_INVALID_ARG),         # the combine writes out
+    (2, 0xB0000, 0xC0000, dict(part_o=0xB0000, part_lse=0xC0000), B.HRA_ERR_WORKSPACE),  # ignored
+    (64, 0xB0000, 0xC0000, {}, B.HRA_ERR_WORKSPACE),                      # well formed: stops at the workspace
+])
+def test_combine_partials_is_validated(n_parts, parts_o, parts_lse, over, status):
+    p = _fake_params(**over)
+    lib = hra.load_library()
+    rc = lib.hra_combine_partials(ctypes.byref(p), n_parts, parts_o, parts_lse, None)
+    assert rc == status, hra.last_error()
+
+
+def test_make_params_sets_the_token_range_fields():
+    import torch
+    q = torch.zeros(1, 4, 192, dtype=torch.bfloat16)
+    cache = torch.zeros(64, 576, dtype=torch.bfloat16)
+    w = torch.zeros(4, 512, 128, dtype=torch.bfloat16)
+    pos = torch.tensor([99], dtype=torch.int32)
+    po = torch.zeros(1, 4, 512)
+    pl = torch.zeros(1, 4, 4)
+    p = hra.make_params(q, cache[:, :512], cache[:, 512:], torch.tensor([64], dtype=torch.int32), w, w, None,
+                        n_branch=4, q_positions=pos, part_o=po, part_lse=pl)
+    assert (p.q_positions, p.part_o, p.part_lse) == (pos.data_ptr(), po.data_ptr(), pl.data_ptr())
+    assert p.out is None
