@@ -607,6 +607,102 @@ def prefill_flops(L: int, n: int, heads: int, n_branch: int = 4) -> int:
     return 4 * L * 512 * 128 * heads + 2 * (192 + 128) * pairs * heads * n_branch
 
 
+def run_cp_bench(args, wl, world, rank, local):
+    """One batch of sequences split over `args.cp` devices by token range: each rank decodes
+    its range into partial states, the states are all-gathered (NCCL) and every rank merges
+    them and finishes the decode.  On one GPU, rank 0 runs alone with its own state standing
+    in for the others' (no all-gather)."""
+    import head_rank_attention_b200 as hra
+    from head_rank_attention_b200 import cp
+    torch.cuda.set_device(local)
+    W = args.cp
+    inp = synth.make_inputs(wl)
+    lengths = [int(x) for x in inp.seq_lens]
+    starts, counts = cp.token_ranges(lengths, rank, W)
+    T = max(max(counts), 1)
+    local_cache = torch.zeros(wl.batch * T, inp.cache.shape[1], dtype=inp.cache.dtype, device="cuda")
+    for s in range(wl.batch):
+        rows = synth.logical_rows(inp, wl, s)[starts[s]:starts[s] + counts[s]]
+        local_cache[s * T:s * T + counts[s]] = rows.cuda()
+    q = inp.q.cuda()
+    w_uk, w_uv = inp.w_uk.cuda(), inp.w_uv.cuda()
+    seq_lens = torch.tensor(counts, dtype=torch.int32, device="cuda")
+    q_pos = torch.tensor([max(n - 1, 0) for n in lengths], dtype=torch.int32, device="cuda")
+    part_o = torch.zeros(wl.batch, wl.heads, synth.D_C, device="cuda")
+    part_lse = torch.zeros(wl.batch, wl.heads, synth.D_C // 128, device="cuda")
+    kw = dict(n_branch=wl.n_branch, alpha_q=wl.alpha_q, alpha_kv=wl.alpha_kv, branch_scale=wl.sigma_o,
+              softmax_scale=wl.softmax_scale, rope_theta=wl.rope_theta)
+    p = hra.make_params(q, local_cache[:, :synth.D_C], local_cache[:, synth.D_C:], seq_lens, w_uk, w_uv, None,
+                        seq_stride=T, q_positions=q_pos, part_o=part_o, part_lse=part_lse, **kw)
+    ws = hra.alloc_workspace(p)
+    out = torch.empty(wl.batch, wl.heads, synth.D_V, dtype=torch.float32, device="cuda")
+    pc = hra.make_params(q, local_cache[:, :synth.D_C], local_cache[:, synth.D_C:], seq_lens, w_uk, w_uv, out,
+                         seq_stride=T, **kw)
+    ws_c = hra.alloc_workspace(pc)
+    stream = torch.cuda.current_stream()
+    if world > 1:
+        gather = lambda: cp.gather_partials(part_o, part_lse)  # noqa: E731
+    else:
+        stand_o = part_o.unsqueeze(0).expand(W, *part_o.shape)
+        stand_l = part_lse.unsqueeze(0).expand(W, *part_lse.shape)
+        gather = lambda: (stand_o.contiguous(), stand_l.contiguous())  # noqa: E731
+
+    def one_step():
+        hra.mlra_decode(p, stream)
+        go, gl = gather()
+        hra.combine_partials(pc, go, gl, stream)
+
+    for _ in range(args.warmup):
+        one_step()
+    hra.check_device_status(p, stream)
+    hra.check_device_status(pc, stream)
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
+           torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    with ClockSampler(torch.cuda.current_device()) as clk:
+        for e0, e1, e2 in ev:
+            e0.record(stream)
+            hra.mlra_decode(p, stream)
+            e1.record(stream)
+            go, gl = gather()
+            hra.combine_partials(pc, go, gl, stream)
+            e2.record(stream)
+        torch.cuda.synchronize()
+    hra.check_device_status(pc, stream)
+    step_ms = statistics.median(e0.elapsed_time(e2) for e0, _, e2 in ev)
+    range_ms = statistics.median(e0.elapsed_time(e1) for e0, e1, _ in ev)
+    step_ms, range_ms = max_over_ranks([step_ms, range_ms], world, "cuda")
+    if rank != 0:
+        return
+    range_bytes = 1152 * sum(counts)
+    all_bytes = 1152 * sum(lengths)
+    done = all_bytes if world == W else range_bytes  # the tokens this job decoded
+    pk, pk_src = peaks()
+    line = {
+        "metric": f"MLRA decode us/step with each sequence split by token range over {W} devices",
+        "value": done / (step_ms * 1e-3) / 1e12, "unit": "TB/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": step_ms, "us_per_step": step_ms * 1e3, "higher_is_better": True,
+        "scaling": "strong", "vs_baseline": None, "dtype": "f16", "data": "synthetic",
+        "config": {"workload": wl.name, "split": W, "tokens_per_rank": counts,
+                   "parallelism": (f"cp{W}: NCCL all-gather of the partial states" if world == W else
+                                   f"cp{W}: rank 0's range alone, its state standing in for the other ranks' "
+                                   f"(no all-gather)"),
+                   "l2": "the range's cache is larger than L2 (no flush)" if range_bytes > (126 << 20)
+                         else "the range's cache fits in L2 (no flush: a lower bound on the time)"},
+        "stage_us": {"range_decode": range_ms * 1e3, "gather_and_combine": (step_ms - range_ms) * 1e3},
+        "roofline": {"bound": "hbm", "achieved": range_bytes / (range_ms * 1e-3) / 1e9, "peak": pk["hbm_gbs"],
+                     "unit": "GB/s", "frac": range_bytes / (range_ms * 1e-3) / 1e9 / pk["hbm_gbs"],
+                     "peak_source": pk_src, "traffic": None,
+                     "note": "the range's KV bytes over the whole range call (absorb, decode, merge)"},
+        "clocks": clk.summary(),
+        "e2e": None,
+        "gpu_launches": 5 * args.steps,  # absorb, decode, merge; partial combine, up-projection
+    }
+    print(json.dumps(line), flush=True)
+
+
 def run_prefill_bench(args, world, rank, local):
     """Prefill of one MLRA-4 sequence (h = 128): the three kernels of mlra_prefill per step."""
     import head_rank_attention_b200 as hra
@@ -729,6 +825,8 @@ def main():
     ap.add_argument("--gla", type=int, default=0, choices=[0, 2],
                     help="a rank of GLA-2 on an MLA workload (2 latent groups, half the heads each)")
     ap.add_argument("--prefill", type=int, default=0, help="time the prefill path over this many cached tokens")
+    ap.add_argument("--cp", type=int, default=0,
+                    help="split every sequence over this many devices by token range (rank 0 alone on one GPU)")
     ap.add_argument("--prefill-queries", type=int, default=0, help="query tokens of --prefill (default: all)")
     args = ap.parse_args()
     if args.warmup < 3:
@@ -759,6 +857,13 @@ def main():
                                                                   "sample is reported as cpu_baseline"}))
             return
         run_prefill_bench(args, world, rank, local)
+    elif args.cp:
+        if args.impl == "reference":
+            print(json.dumps({"impl": "reference", "unavailable": "the token-range split has no reference arm"}))
+            return
+        if world not in (1, args.cp) or args.tp or args.gla or args.cache != "bf16" or wl.page_size:
+            ap.error(f"--cp {args.cp} runs on {args.cp} ranks (or one GPU), bf16, contiguous, no --tp / --gla")
+        run_cp_bench(args, wl, world, rank, local)
     elif args.impl == "reference":
         run_reference(args, wl, world, rank)
     else:
