@@ -858,11 +858,11 @@ def main():
             return
         run_prefill_bench(args, world, rank, local)
     elif args.cp:
+        if world not in (1, args.cp) or args.tp or args.gla or args.cache != "bf16" or wl.page_size:
+            ap.error(f"--cp {args.cp} runs on {args.cp} ranks (or one GPU), bf16, contiguous, no --tp / --gla")
         if args.impl == "reference":
             print(json.dumps({"impl": "reference", "unavailable": "the token-range split has no reference arm"}))
             return
-        if world not in (1, args.cp) or args.tp or args.gla or args.cache != "bf16" or wl.page_size:
-            ap.error(f"--cp {args.cp} runs on {args.cp} ranks (or one GPU), bf16, contiguous, no --tp / --gla")
         run_cp_bench(args, wl, world, rank, local)
     elif args.impl == "reference":
         run_reference(args, wl, world, rank)

@@ -178,3 +178,23 @@ def test_recorded_traffic_is_keyed_by_shard_group_and_cache_format(tmp_path):
     assert bench.ncu_traffic(bench.traffic_key("w"), f) == 123
     assert bench.ncu_traffic(bench.traffic_key("w", int8=True), f) is None   # stale source
     assert bench.ncu_traffic(bench.traffic_key("w", tp=4), f) is None        # not recorded
+
+
+@pytest.mark.parametrize("extra", [["--tp", "4"], ["--workload", "paged_b64_t32k_mlra4"], ["--cache", "int8"]])
+def test_token_range_split_mode_refuses_other_layouts(extra):
+    """--cp W takes contiguous bf16 workloads without --tp / --gla; the rest is refused
+    before any device work."""
+    import subprocess
+    args = ["--cp", "2", "--workload", "long_mlra4_b4_t64k_128k"] + extra
+    r = subprocess.run(_bench_cmd(*args), capture_output=True, text=True, timeout=300)
+    assert r.returncode == 2 and "--cp 2" in r.stderr, r.stderr[-300:]
+
+
+def test_token_range_split_has_no_reference_arm():
+    import json
+    import subprocess
+    r = subprocess.run(_bench_cmd("--cp", "2", "--workload", "long_mlra4_b4_t64k_128k", "--impl", "reference"),
+                       capture_output=True, text=True, timeout=300)
+    assert r.returncode == 0
+    line = json.loads([x for x in r.stdout.splitlines() if x.startswith("{")][0])
+    assert line["impl"] == "reference" and "unavailable" in line
